@@ -1,0 +1,6 @@
+"""Float64 CPU oracle for scaled dot-product attention (test infrastructure only).
+
+Only tests, the smoke check and the benchmark's CPU-baseline legs may import
+this package; the product path never does.
+"""
+from .sdpa_ref import default_scale, sdpa, sdpa_packed  # noqa: F401
