@@ -1,0 +1,147 @@
+/*
+ * sdpa15.h -- C ABI of a B200 (sm_100a) scaled dot-product attention forward.
+ *
+ * The operation (exactref.ai, "scaled_dot_product_attention", sections
+ * "Arguments" and "Full specification"):
+ *
+ *     O   = softmax(Q K^T * scale + mask) V        over the key axis
+ *     lse = log(sum_j exp(logit_ij))               natural log, per query row
+ *
+ * - scale: when has_scale == 0 it is 1/sqrt(E), applied exactly once to the
+ *   raw dot products; an explicit scale (e.g. 1/E, or 1.0 for a query that was
+ *   pre-scaled by the caller) is used as given.  Pre-scaling Q and also taking
+ *   the default gives the double-scaled 1/E attention of the hourtab.com
+ *   xFormers post ("Why double scaling makes attention uniform").
+ * - mask kinds: NONE; CAUSAL keeps key j for query i iff j <= i (top-left
+ *   aligned when L != S); BLOCK_DIAG / BLOCK_DIAG_CAUSAL restrict every query
+ *   of a packed batch to the keys of its own segment (xFormers
+ *   BlockDiagonalMask / BlockDiagonalCausalMask, insureai360 tutorial section
+ *   4 "Variable-length packed batch"); FLOAT_BIAS adds a float32 bias to the
+ *   scaled scores, -inf removing a key.  A bool mask is passed as a 0/-inf bias.
+ * - GQA (exactref "Arguments", enable_gqa; the BMGHK layout of the tutorial's
+ *   section 5): Hq is a multiple of Hkv and query head h reads key/value head
+ *   h / (Hq / Hkv).
+ * - lse is float32 for every input dtype (the compute format of the output:
+ *   float32 for formats narrower than float32, exactref "logsumexp and its
+ *   format").  A row with no kept key has O = 0 and lse = -inf; a NaN input
+ *   makes its row NaN (exactref "Special values and dropout").
+ *
+ * Memory and threading contract of every entry point below:
+ * - All tensor pointers are DEVICE pointers on the current CUDA device.  The
+ *   caller owns and allocates every buffer, the workspace included; the
+ *   library allocates no device memory on this path and never synchronises:
+ *   work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *   stream) and the call returns once it is enqueued.
+ * - Strides are in ELEMENTS, four per tensor, in the order
+ *   (batch, head, sequence, feature).  BHLE (B,H,L,E) and BMHK (B,M,H,K)
+ *   layouts are both expressed this way.  The feature stride must be 1.
+ * - Errors are returned as sdpa_status codes; nothing traps or aborts.  On an
+ *   error no work has been enqueued, except SDPA_ERR_CUDA, which reports a
+ *   failed launch.
+ */
+#ifndef SDPA15_H
+#define SDPA15_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SDPA_OK = 0,
+  SDPA_ERR_INVALID = 1,     /* bad argument: null pointer, shape, stride, GQA ratio, cu_seqlens, dtype */
+  SDPA_ERR_UNSUPPORTED = 2, /* well-formed but not implemented: E or Ev outside 1..256, not an sm_100 device */
+  SDPA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  SDPA_ERR_WORKSPACE = 4    /* workspace missing or smaller than sdpa_fwd_workspace_size() */
+} sdpa_status;
+
+typedef enum { SDPA_F32 = 0, SDPA_F16 = 1, SDPA_BF16 = 2 } sdpa_dtype;
+
+typedef enum {
+  SDPA_MASK_NONE = 0,
+  SDPA_MASK_CAUSAL = 1,
+  SDPA_MASK_BLOCK_DIAG = 2,
+  SDPA_MASK_BLOCK_DIAG_CAUSAL = 3,
+  SDPA_MASK_FLOAT_BIAS = 4
+} sdpa_mask_kind;
+
+/* Version of this ABI (changes when a signature or an enum changes). */
+int sdpa_abi_version(void);
+
+/* Human-readable name of a status code (a static string; never NULL). */
+const char* sdpa_status_string(int status);
+
+/*
+ * Bytes of device workspace sdpa_fwd() needs for this problem (0 when it needs
+ * none).  Depends only on the arguments; the same arguments always give the
+ * same size.  Pass a workspace of at least this many bytes, 256-byte aligned.
+ * Returns 0 for arguments sdpa_fwd() would reject.
+ */
+size_t sdpa_fwd_workspace_size(int B, int Hq, int Hkv, int L, int S, int E, int Ev,
+                               int mask_kind, int dtype);
+
+/*
+ * Attention forward: out = softmax(q k^T * scale + mask) v, lse = per-row
+ * logsumexp of the logits.
+ *
+ * q     [B, Hq,  L, E ]  dtype, strides q_stride   (elements)
+ * k     [B, Hkv, S, E ]  dtype, strides k_stride
+ * v     [B, Hkv, S, Ev]  dtype, strides v_stride
+ * out   [B, Hq,  L, Ev]  dtype, strides o_stride   (written)
+ * lse   [B, Hq,  L]      float32, contiguous       (written)
+ * dtype             SDPA_F32, SDPA_F16 or SDPA_BF16 (q, k, v and out share it)
+ * has_scale, scale  has_scale == 0: scale = 1/sqrt(E); else `scale` as given
+ *                   (any finite value, 0 included)
+ * mask_kind         sdpa_mask_kind
+ * cu_seqlens        BLOCK_DIAG*: device int32[n_seqs + 1], cumulative segment
+ *                   starts of one packed batch: cu[0] = 0, non-decreasing,
+ *                   cu[n_seqs] = L = S, and B must be 1.  Otherwise ignored.
+ *                   The kernels clamp every segment to [0, L), so a malformed
+ *                   array cannot make them read or write out of bounds.
+ * n_seqs            number of segments (>= 1) for BLOCK_DIAG*
+ * max_seqlen        BLOCK_DIAG*: an upper bound on the segment lengths (the
+ *                   grid is sized from it; segments longer than it are an
+ *                   error the kernels cannot detect and leave rows unwritten)
+ * bias, bias_stride FLOAT_BIAS: device float32 [B, Hq, L, S] with element
+ *                   strides (b, h, l, s); 0 broadcasts an axis.  Else ignored.
+ * workspace         device scratch of sdpa_fwd_workspace_size() bytes (may be
+ *                   NULL when that size is 0); its contents need no clearing
+ *                   and are garbage afterwards.
+ * stream            cudaStream_t to enqueue on.
+ *
+ * Returns SDPA_OK or an error status (see sdpa_status).
+ */
+int sdpa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+             int B, int Hq, int Hkv, int L, int S, int E, int Ev,
+             const int64_t q_stride[4], const int64_t k_stride[4],
+             const int64_t v_stride[4], const int64_t o_stride[4],
+             int has_scale, float scale,
+             int mask_kind, const int32_t* cu_seqlens, int n_seqs, int max_seqlen,
+             const float* bias, const int64_t bias_stride[4],
+             int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Which kernel family sdpa_fwd() would run for these arguments (no work is
+ * done): 1 = tcgen05/TMA prefill, 2 = split-S decode + combine, 3 = general
+ * SIMT kernel, or a negative sdpa_status for rejected arguments.  For tests
+ * and benchmarks that must know the path taken.
+ */
+int sdpa_fwd_plan(int B, int Hq, int Hkv, int L, int S, int E, int Ev,
+                  const int64_t q_stride[4], const int64_t k_stride[4],
+                  const int64_t v_stride[4], const int64_t o_stride[4],
+                  int mask_kind, int dtype,
+                  const void* q, const void* k, const void* v, const void* out);
+
+/*
+ * Number of kernels the last successful sdpa_fwd() call on this host thread
+ * enqueued (1 or 2), for launch accounting in benchmarks.
+ */
+int sdpa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA15_H */

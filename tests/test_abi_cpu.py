@@ -1,0 +1,109 @@
+"""CPU checks of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before touching a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from scaled_dot_product_15_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sdpa15.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sdpa_\w+)\s*\(", src)))
+
+
+def test_header_declares_bound_symbols():
+    assert _declared() == sorted(api.exported_symbols())
+
+
+def test_library_exports_every_declared_symbol():
+    lib = api.load_library()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", api.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (sdpa_\w+)$", out, flags=re.M))
+    assert set(_declared()) <= exported
+
+
+def test_status_strings_and_version():
+    lib = api.load_library()
+    assert lib.sdpa_abi_version() == 1
+    for s in range(5):
+        assert lib.sdpa_status_string(s)
+    assert lib.sdpa_status_string(99) == b"unknown status"
+
+
+def _call(**kw):
+    lib = api.load_library()
+    a = dict(B=1, Hq=2, Hkv=2, L=8, S=8, E=64, Ev=64, mask=0, dtype=api.SDPA_BF16, scale=None,
+             cu=None, n_seqs=0, maxlen=0, bias=None, ws=None, ws_bytes=0)
+    a.update(kw)
+    fake = 0x10000  # never dereferenced: every case below fails on the host
+    st = api._i64x4((a["Hq"] * a["L"] * a["E"], a["L"] * a["E"], a["E"], 1))
+    sv = api._i64x4((a["Hkv"] * a["S"] * a["Ev"], a["S"] * a["Ev"], a["Ev"], 1))
+    sk = api._i64x4((a["Hkv"] * a["S"] * a["E"], a["S"] * a["E"], a["E"], 1))
+    so = api._i64x4((a["Hq"] * a["L"] * a["Ev"], a["L"] * a["Ev"], a["Ev"], 1))
+    if "qstride" in kw:
+        st = api._i64x4(kw["qstride"])
+    ptr = kw.get("ptr", fake)
+    return lib.sdpa_fwd(ptr, fake, fake, fake, fake, a["B"], a["Hq"], a["Hkv"], a["L"], a["S"], a["E"], a["Ev"],
+                        st, sk, sv, so, 0 if a["scale"] is None else 1, a["scale"] or 0.0, a["mask"], a["cu"],
+                        a["n_seqs"], a["maxlen"], a["bias"], api._i64x4((0, 0, 0, 0)), a["dtype"], a["ws"],
+                        a["ws_bytes"], None)
+
+
+def test_host_side_rejections():
+    assert _call(Hq=3, Hkv=2) == api.SDPA_ERR_INVALID          # Hq not a multiple of Hkv
+    assert _call(dtype=7) == api.SDPA_ERR_INVALID               # unknown dtype
+    assert _call(mask=9) == api.SDPA_ERR_INVALID                # unknown mask
+    assert _call(E=0) == api.SDPA_ERR_UNSUPPORTED               # E = 0 is not run on the GPU
+    assert _call(E=512) == api.SDPA_ERR_UNSUPPORTED
+    assert _call(qstride=(1, 1, 1, 2)) == api.SDPA_ERR_INVALID  # feature stride must be 1
+    assert _call(mask=api.MASK_BLOCK_DIAG, B=2) == api.SDPA_ERR_INVALID
+    assert _call(mask=api.MASK_BLOCK_DIAG) == api.SDPA_ERR_INVALID  # no cu_seqlens
+    assert _call(mask=api.MASK_FLOAT_BIAS) == api.SDPA_ERR_INVALID  # no bias
+    assert _call(scale=float("nan")) == api.SDPA_ERR_INVALID
+    assert _call(ptr=None) == api.SDPA_ERR_INVALID
+    assert _call(B=0) == api.SDPA_OK                            # empty problem: nothing to do
+    assert _call(L=0) == api.SDPA_OK
+
+
+def test_no_gpu_means_unsupported_not_a_crash():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _call() == api.SDPA_ERR_UNSUPPORTED
+
+
+def test_workspace_size_is_deterministic():
+    lib = api.load_library()
+    args = (64, 32, 8, 1, 16384, 128, 128, api.MASK_NONE, api.SDPA_BF16)
+    n = lib.sdpa_fwd_workspace_size(*args)
+    assert n > 0 and n == lib.sdpa_fwd_workspace_size(*args)
+    assert n % 4 == 0
+    assert lib.sdpa_fwd_workspace_size(4, 16, 16, 2048, 2048, 128, 128, api.MASK_CAUSAL, api.SDPA_BF16) == 0
+    assert lib.sdpa_fwd_workspace_size(1, 3, 2, 1, 10, 64, 64, 0, api.SDPA_BF16) == 0  # invalid
+
+
+def _plan(B, Hq, Hkv, L, S, E, Ev, mask, dtype, align=0):
+    lib = api.load_library()
+    st = lambda H, n, e: api._i64x4((H * n * e, n * e, e, 1))
+    base = 0x100000 + align
+    return lib.sdpa_fwd_plan(B, Hq, Hkv, L, S, E, Ev, st(Hq, L, E), st(Hkv, S, E), st(Hkv, S, Ev),
+                             st(Hq, L, Ev), mask, dtype, base, base, base, base)
+
+
+def test_dispatch_plan():
+    assert _plan(1, 2, 2, 64, 64, 16, 16, 0, api.SDPA_F32) == 3              # fp32: SIMT
+    assert _plan(64, 32, 8, 1, 16384, 128, 128, 0, api.SDPA_BF16) == 2       # GQA decode
+    assert _plan(64, 32, 8, 1, 16384, 128, 128, 0, api.SDPA_BF16, align=2) == 3  # unaligned
+    assert _plan(1, 2, 2, 64, 64, 48, 48, api.MASK_FLOAT_BIAS, api.SDPA_F16) == 3
+    assert _plan(1, 3, 2, 64, 64, 64, 64, 0, api.SDPA_F16) == -api.SDPA_ERR_INVALID

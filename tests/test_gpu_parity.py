@@ -1,0 +1,287 @@
+"""Parity of the CUDA library with the float64 oracle on the same seeded inputs.
+
+Tolerances (stated for the method): float32 max |diff| <= 1e-5 * max(1, max|ref|)
+on O and on lse; bf16/fp16 max |diff| <= 2e-2 on O and <= 1e-2 on lse.  NaN
+and infinity positions must agree exactly.
+
+Small cases are compared element by element; the full-size workloads, in the
+launch configuration the benchmark times, on sampled rows that the oracle
+computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import sdpa as ref_sdpa
+from oracle import sdpa_packed as ref_packed
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+O_TOL = {torch.float16: 2e-2, torch.bfloat16: 2e-2}
+L_TOL = {torch.float16: 1e-2, torch.bfloat16: 1e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from scaled_dot_product_15_b200 import api, build
+
+    import os
+
+    if not os.path.exists(api.LIB_PATH):
+        build.build()
+    api.load_library()
+    assert torch.cuda.is_available(), "these tests need a GPU"
+
+
+def _sdpa(*a, **k):
+    from scaled_dot_product_15_b200 import sdpa
+
+    out, lse = sdpa(*a, **k)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def _plan(*a, **k):
+    from scaled_dot_product_15_b200 import plan
+
+    return plan(*a, **k)
+
+
+def assert_close(out, lse, ref_o, ref_l, dtype, what=""):
+    got_o = out.detach().double().cpu().numpy() if torch.is_tensor(out) else np.asarray(out)
+    got_l = lse.detach().double().cpu().numpy() if torch.is_tensor(lse) else np.asarray(lse)
+    ref_o = np.asarray(ref_o, dtype=np.float64)
+    ref_l = np.asarray(ref_l, dtype=np.float64)
+    assert got_o.shape == ref_o.shape, (got_o.shape, ref_o.shape)
+    assert got_l.shape == ref_l.shape, (got_l.shape, ref_l.shape)
+    for g, r, name in ((got_o, ref_o, "O"), (got_l, ref_l, "lse")):
+        assert np.array_equal(np.isnan(g), np.isnan(r)), f"{what} {name}: NaN positions differ"
+        fin = np.isfinite(r)
+        assert np.array_equal(g[~fin & ~np.isnan(r)], r[~fin & ~np.isnan(r)]), f"{what} {name}: inf differ"
+    fo, fl = np.isfinite(ref_o), np.isfinite(ref_l)
+    if dtype == torch.float32:
+        to = 1e-5 * max(1.0, np.abs(ref_o[fo]).max(initial=0.0))
+        tl = 1e-5 * max(1.0, np.abs(ref_l[fl]).max(initial=0.0))
+    else:
+        to, tl = O_TOL[dtype], L_TOL[dtype]
+    eo = np.abs(got_o[fo] - ref_o[fo]).max(initial=0.0)
+    el = np.abs(got_l[fl] - ref_l[fl]).max(initial=0.0)
+    assert eo <= to, f"{what}: max |dO| = {eo:.3e} > {to:.1e}"
+    assert el <= tl, f"{what}: max |dlse| = {el:.3e} > {tl:.1e}"
+    return eo, el
+
+
+def _rand(shape, seed, dtype):
+    return W.randn(shape, seed, dtype)
+
+
+# ---------------------------------------------------------------- small, full compare
+
+
+@pytest.mark.parametrize("name", ["fp32_b1_h2_l64_e16", "fp32_b1_h2_l64_e16_causal"])
+def test_fp32_small_workload(name):
+    w = W.WORKLOADS[name]
+    q, k, v = W.make_inputs(w)
+    for _ in range(2):  # run twice: same result
+        out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), is_causal=w.mask == "causal")
+        ro, rl = ref_sdpa(q, k, v, is_causal=w.mask == "causal")
+        assert_close(out, lse, ro, rl, torch.float32, name)
+
+
+PREFILL_CASES = [
+    # dtype, B, Hq, Hkv, L, S, E, Ev, causal
+    (torch.bfloat16, 1, 2, 2, 300, 300, 128, 128, True),
+    (torch.bfloat16, 2, 2, 2, 256, 256, 128, 128, False),
+    (torch.float16, 1, 2, 2, 200, 333, 64, 64, False),
+    (torch.float16, 1, 2, 2, 257, 257, 96, 96, True),
+    (torch.float16, 1, 3, 3, 129, 129, 64, 64, True),
+    (torch.bfloat16, 1, 8, 2, 200, 200, 128, 128, True),   # GQA prefill
+    (torch.bfloat16, 1, 2, 2, 300, 100, 128, 128, True),   # L > S: rows past S keep all keys
+    (torch.float16, 1, 2, 2, 17, 400, 96, 96, False),
+    (torch.bfloat16, 1, 2, 2, 70, 70, 32, 48, False),     # odd head sizes: general kernel
+    (torch.float32, 1, 2, 2, 100, 77, 40, 24, True),
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=lambda c: "-".join(str(x) for x in c))
+def test_prefill_small(case):
+    dt, B, Hq, Hkv, L, S, E, Ev, causal = case
+    q = _rand((B, Hq, L, E), 101, dt)
+    k = _rand((B, Hkv, S, E), 102, dt)
+    v = _rand((B, Hkv, S, Ev), 103, dt)
+    out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), is_causal=causal, enable_gqa=Hq != Hkv)
+    ro, rl = ref_sdpa(q, k, v, is_causal=causal, enable_gqa=Hq != Hkv)
+    assert_close(out, lse, ro, rl, dt, str(case))
+
+
+DECODE_CASES = [
+    # dtype, B, Hq, Hkv, L, S, E
+    (torch.bfloat16, 2, 8, 2, 1, 3000, 128),
+    (torch.float16, 3, 4, 4, 1, 100, 64),
+    (torch.bfloat16, 1, 8, 1, 1, 5000, 256),
+    (torch.float16, 2, 8, 2, 2, 1025, 128),     # 8 rows per key head
+    (torch.bfloat16, 1, 2, 1, 1, 1, 128),       # one cached key
+    (torch.bfloat16, 1, 1, 1, 3, 20000, 64),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=lambda c: "-".join(str(x) for x in c))
+def test_decode_small(case):
+    dt, B, Hq, Hkv, L, S, E = case
+    q = _rand((B, Hq, L, E), 201, dt)
+    k = _rand((B, Hkv, S, E), 202, dt)
+    v = _rand((B, Hkv, S, E), 203, dt)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    assert _plan(qd, kd, vd) == "decode_split"
+    out, lse = _sdpa(qd, kd, vd, enable_gqa=Hq != Hkv)
+    ro, rl = ref_sdpa(q, k, v, enable_gqa=Hq != Hkv)
+    assert_close(out, lse, ro, rl, dt, str(case))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dt,E", [(torch.float16, 64), (torch.bfloat16, 128), (torch.float16, 96)])
+def test_varlen_small(causal, dt, E):
+    seqlens = [5, 130, 1, 257, 64, 300, 128]
+    T, H = sum(seqlens), 2
+    q = _rand((1, T, H, E), 301, dt)
+    k = _rand((1, T, H, E), 302, dt)
+    v = _rand((1, T, H, E), 303, dt)
+    cu = torch.tensor(W.cu_seqlens_of(seqlens), dtype=torch.int32, device=DEV)
+    out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), is_causal=causal, cu_seqlens=cu, max_seqlen=max(seqlens))
+    ro, rl = ref_packed(q, k, v, seqlens, causal=causal)
+    assert_close(out, lse[0], ro, rl, dt, f"varlen causal={causal}")
+
+
+def test_bmhk_layout_and_strided_views():
+    dt = torch.bfloat16
+    q = _rand((2, 150, 4, 128), 401, dt)
+    k = _rand((2, 150, 4, 128), 402, dt)
+    v = _rand((2, 150, 4, 128), 403, dt)
+    out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), is_causal=True, layout="bmhk")
+    ro, rl = ref_sdpa(q.transpose(1, 2), k.transpose(1, 2), v.transpose(1, 2), is_causal=True)
+    assert_close(out.transpose(1, 2), lse, ro, rl, dt, "bmhk")
+    # BHLE views of the same memory (non-contiguous strides)
+    out2, lse2 = _sdpa(q.to(DEV).transpose(1, 2), k.to(DEV).transpose(1, 2), v.to(DEV).transpose(1, 2),
+                       is_causal=True)
+    assert_close(out2, lse2, ro, rl, dt, "bhle view")
+
+
+def test_masks_and_special_values():
+    dt = torch.float16
+    B, H, L, S, E = 1, 2, 40, 50, 64
+    q = _rand((B, H, L, E), 501, dt)
+    k = _rand((B, H, S, E), 502, dt)
+    v = _rand((B, H, S, E), 503, dt)
+    g = torch.Generator().manual_seed(504)
+    bias = torch.randn(B, 1, L, S, generator=g)
+    bias[..., 7] = float("-inf")
+    bias[0, 0, 3, :] = float("-inf")       # a row with no kept key
+    out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), attn_mask=bias.to(DEV))
+    ro, rl = ref_sdpa(q, k, v, attn_mask=bias)
+    assert_close(out, lse, ro, rl, dt, "float bias")
+    assert (out[0, :, 3] == 0).all() and torch.isneginf(lse[0, :, 3]).all()
+    boolm = torch.rand(L, S, generator=g) > 0.5
+    boolm[5] = False
+    out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), attn_mask=boolm.to(DEV))
+    ro, rl = ref_sdpa(q, k, v, attn_mask=boolm)
+    assert_close(out, lse, ro, rl, dt, "bool mask")
+    qn = q.clone()
+    qn[0, 1, 9, 0] = float("nan")
+    out, lse = _sdpa(qn.to(DEV), k.to(DEV), v.to(DEV))
+    ro, rl = ref_sdpa(qn, k, v)
+    assert_close(out, lse, ro, rl, dt, "NaN row")
+    assert torch.isnan(out[0, 1, 9]).all()
+
+
+@pytest.mark.parametrize("scale", [1.0, 1.0 / 96, 0.0])
+def test_explicit_scales(scale):
+    dt = torch.float16
+    q = _rand((1, 2, 130, 96), 601, dt)
+    k = _rand((1, 2, 130, 96), 602, dt)
+    v = _rand((1, 2, 130, 96), 603, dt)
+    out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), is_causal=True, scale=scale)
+    ro, rl = ref_sdpa(q, k, v, is_causal=True, scale=scale)
+    assert_close(out, lse, ro, rl, dt, f"scale={scale}")
+
+
+def test_dropout_and_dtype_errors():
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.float16, device=DEV)
+    with pytest.raises(ValueError, match="dropout_p must be 0"):
+        _sdpa(q, q, q, dropout_p=0.1)
+    with pytest.raises(ValueError):
+        _sdpa(q, q.to(torch.bfloat16), q)
+
+
+# ---------------------------------------------------------------- full sizes, sampled
+
+
+def _causal_rows_bias(rows, S):
+    j = np.arange(S)[None, :]
+    return np.where(j <= np.asarray(rows)[:, None], 0.0, -np.inf)
+
+
+def _sampled_prefill_check(w, samples, rows):
+    q, k, v = W.make_inputs(w, DEV)
+    causal = w.mask == "causal"
+    out, lse = _sdpa(q, k, v, is_causal=causal, scale=w.scale)
+    worst = (0.0, 0.0)
+    for b, h in samples:
+        qs = W.make_slice(w, "q", b)[h][rows][None, None]
+        ks = W.make_slice(w, "k", b)[h // (w.Hq // w.Hkv)][None, None]
+        vs = W.make_slice(w, "v", b)[h // (w.Hq // w.Hkv)][None, None]
+        bias = _causal_rows_bias(rows, w.S) if causal else None
+        ro, rl = ref_sdpa(qs, ks, vs, attn_mask=bias, scale=w.scale)
+        e = assert_close(out[b, h, rows][None, None], lse[b, h, rows][None, None], ro, rl, w.torch_dtype,
+                         f"{w.name} b={b} h={h}")
+        worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+    return out, lse, worst
+
+
+ROWS_2048 = [0, 1, 2, 63, 127, 128, 129, 255, 511, 1000, 1023, 1024, 1500, 2046, 2047]
+
+
+def test_full_bf16_causal_prefill_sampled():
+    w = W.WORKLOADS["bf16_causal_b4_h16_l2048_e128"]
+    _sampled_prefill_check(w, [(0, 0), (1, 7), (3, 15)], ROWS_2048)
+
+
+@pytest.mark.parametrize("name", ["fp16_causal_b1_h64_l2048_e96", "fp16_causal_b1_h64_l2048_e96_scale1_96"])
+def test_full_fp16_hd96_sampled(name):
+    w = W.WORKLOADS[name]
+    out, lse, _ = _sampled_prefill_check(w, [(0, 0), (0, 31), (0, 63)], ROWS_2048)
+    if w.scale is not None:
+        # double-scaled: near-uniform weights, lse ~ log(i+1) + (small)
+        i = torch.arange(2048, device=DEV, dtype=torch.float32)
+        gap = (lse[0] - torch.log(i + 1)).abs()
+        assert gap[:, 1:].max().item() < 0.05
+
+
+def test_full_fp16_varlen_sampled():
+    w = W.WORKLOADS["fp16_varlen_t32768_h8_e64"]
+    seqlens = W.workload_seqlens(w)
+    q, k, v = W.make_inputs(w, DEV)
+    cu = torch.tensor(W.cu_seqlens_of(seqlens), dtype=torch.int32, device=DEV)
+    out, lse = _sdpa(q, k, v, is_causal=True, cu_seqlens=cu, max_seqlen=max(seqlens))
+    qc, kc, vc = W.make_inputs(w, "cpu")
+    heads = [0, 5]
+    ro, rl = ref_packed(qc, kc, vc, seqlens, causal=True, heads=heads)
+    assert_close(out[:, :, heads], lse[0][heads], ro[:, :, heads], rl[heads], w.torch_dtype, w.name)
+
+
+def test_full_bf16_gqa_decode_sampled():
+    w = W.WORKLOADS["bf16_gqa_decode_b64_hq32_hkv8_s16384_e128"]
+    q, k, v = W.make_inputs(w, DEV)
+    assert _plan(q, k, v) == "decode_split"
+    out, lse = _sdpa(q, k, v, enable_gqa=True)
+    g = w.Hq // w.Hkv
+    for b, kvh in [(0, 0), (17, 3), (63, 7)]:
+        qs = W.make_slice(w, "q", b)[kvh * g:(kvh + 1) * g][None]
+        ks = W.make_slice(w, "k", b)[kvh][None, None]
+        vs = W.make_slice(w, "v", b)[kvh][None, None]
+        ro, rl = ref_sdpa(qs, ks, vs, enable_gqa=True)
+        assert_close(out[b, kvh * g:(kvh + 1) * g][None], lse[b, kvh * g:(kvh + 1) * g][None], ro, rl,
+                     w.torch_dtype, f"decode b={b} kvh={kvh}")
