@@ -180,7 +180,7 @@ def make_sets(w: W.Workload, device):
     """Input sets for a workload: enough copies that their total exceeds L2."""
     q, k, v = W.make_inputs(w, device)
     set_bytes = _bytes_of((q, k, v))
-    n = 1 if set_bytes > 2 * L2_BYTES else int(math.ceil(2.5 * L2_BYTES / set_bytes))
+    n = 1 if set_bytes > 2 * L2_BYTES else min(16, int(math.ceil(2.5 * L2_BYTES / set_bytes)))
     sets = [(q, k, v)]
     for i in range(1, n):
         # different memory, same values: L2 residency is what matters
@@ -327,7 +327,8 @@ def measure_workload(w: W.Workload, steps: int, warmup: int, peaks, peak_src, de
         "path": calls[0].plan,
         "gpu_launches": launches,
         "roofline": roofline(w, kernel_ms, peaks, peak_src),
-        "l2": f"{len(sets)} rotating input sets of {set_bytes / 1e6:.1f} MB",
+        "l2": (f"{len(sets)} rotating input sets of {set_bytes / 1e6:.1f} MB"
+               + (" (all sets fit in L2: latency case)" if len(sets) * set_bytes < L2_BYTES else "")),
     }
     if w.layout == "packed":
         res["flops_exact"] = W.flops(w)

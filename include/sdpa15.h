@@ -140,6 +140,15 @@ int sdpa_fwd_plan(int B, int Hq, int Hkv, int L, int S, int E, int Ev,
  */
 int sdpa_last_launch_count(void);
 
+/*
+ * Reads and clears the device-side error word of the current device
+ * (synchronises the device).  *code receives 0 when no kernel gave up; a
+ * non-zero value means a kernel's bounded wait on one of its own pipeline
+ * barriers ran out (2 s) and its outputs for that launch are not valid.
+ * Returns SDPA_OK, SDPA_ERR_INVALID for a NULL `code`, or SDPA_ERR_CUDA.
+ */
+int sdpa_take_device_error(int* code);
+
 #ifdef __cplusplus
 }
 #endif

@@ -52,6 +52,7 @@ _SIGNATURES = {
         [ctypes.c_int] * 7 + [_I64x4] * 4 + [ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4,
     ),
     "sdpa_last_launch_count": (ctypes.c_int, []),
+    "sdpa_take_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
 }
 
 _lib = None
@@ -252,6 +253,13 @@ def plan(query, key, value, *, layout="bhle", mask_kind=MASK_NONE, out=None) -> 
     if r < 0:
         _check(-r, "sdpa_fwd_plan")
     return PLAN_NAMES[r]
+
+
+def take_device_error() -> int:
+    """Device-side error word (0 = no kernel gave up on a wait), cleared."""
+    code = ctypes.c_int(0)
+    _check(load_library().sdpa_take_device_error(ctypes.byref(code)), "sdpa_take_device_error")
+    return code.value
 
 
 def last_launch_count() -> int:

@@ -13,6 +13,7 @@ cudaError_t launch_decode(const Params& p, int dtype, cudaStream_t st, int* laun
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int L, int S, int Ev);
 bool prefill_supported(const Params& p, int dtype);
 cudaError_t launch_prefill(const Params& p, int dtype, cudaStream_t st);
+cudaError_t prefill_take_error(int* code);
 }  // namespace sdpa15
 
 using namespace sdpa15;
@@ -55,6 +56,8 @@ void fill_params(Params& p, const void* q, const void* k, const void* v, void* o
   p.group = Hq / Hkv;
   for (int d = 0; d < 4; ++d) { p.qs[d] = qs[d]; p.ks[d] = ks[d]; p.vs[d] = vs[d]; p.os[d] = os[d]; }
   p.mask = mask;
+  p.scale = (float)(1.0 / sqrt((double)E));  // the default; sdpa_fwd() sets the real one
+  p.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
 }
 
 int choose_plan(const Params& p, int dtype) {
@@ -92,6 +95,13 @@ const char* sdpa_status_string(int status) {
 }
 
 int sdpa_last_launch_count(void) { return t_last_launches; }
+
+int sdpa_take_device_error(int* code) {
+  if (!code) return SDPA_ERR_INVALID;
+  *code = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SDPA_ERR_CUDA;
+  return prefill_take_error(code) == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
 
 size_t sdpa_fwd_workspace_size(int B, int Hq, int Hkv, int L, int S, int E, int Ev, int mask_kind,
                                int dtype) {

@@ -38,10 +38,11 @@ def _lib():
 
 
 def _sdpa(*a, **k):
-    from scaled_dot_product_15_b200 import sdpa
+    from scaled_dot_product_15_b200 import api, sdpa
 
     out, lse = sdpa(*a, **k)
     torch.cuda.synchronize()
+    assert api.take_device_error() == 0, "a kernel gave up on a bounded wait"
     return out, lse
 
 
@@ -104,6 +105,9 @@ PREFILL_CASES = [
     (torch.float16, 1, 2, 2, 17, 400, 96, 96, False),
     (torch.bfloat16, 1, 2, 2, 70, 70, 32, 48, False),     # odd head sizes: general kernel
     (torch.float32, 1, 2, 2, 100, 77, 40, 24, True),
+    (torch.bfloat16, 1, 2, 2, 1, 300, 128, 128, True),    # one query row: key 0 only
+    (torch.float16, 2, 4, 4, 700, 700, 128, 128, True),   # several 256-row blocks, ragged tail
+    (torch.bfloat16, 1, 2, 2, 513, 1500, 64, 64, False),
 ]
 
 
@@ -113,7 +117,10 @@ def test_prefill_small(case):
     q = _rand((B, Hq, L, E), 101, dt)
     k = _rand((B, Hkv, S, E), 102, dt)
     v = _rand((B, Hkv, S, Ev), 103, dt)
-    out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), is_causal=causal, enable_gqa=Hq != Hkv)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    want = "prefill_tcgen05" if (dt != torch.float32 and E == Ev and E in (64, 96, 128)) else "simt"
+    assert _plan(qd, kd, vd, mask_kind=1 if causal else 0) == want
+    out, lse = _sdpa(qd, kd, vd, is_causal=causal, enable_gqa=Hq != Hkv)
     ro, rl = ref_sdpa(q, k, v, is_causal=causal, enable_gqa=Hq != Hkv)
     assert_close(out, lse, ro, rl, dt, str(case))
 
@@ -227,6 +234,7 @@ def _causal_rows_bias(rows, S):
 def _sampled_prefill_check(w, samples, rows):
     q, k, v = W.make_inputs(w, DEV)
     causal = w.mask == "causal"
+    assert _plan(q, k, v, mask_kind=1 if causal else 0) == "prefill_tcgen05"
     out, lse = _sdpa(q, k, v, is_causal=causal, scale=w.scale)
     worst = (0.0, 0.0)
     for b, h in samples:
@@ -254,10 +262,12 @@ def test_full_fp16_hd96_sampled(name):
     w = W.WORKLOADS[name]
     out, lse, _ = _sampled_prefill_check(w, [(0, 0), (0, 31), (0, 63)], ROWS_2048)
     if w.scale is not None:
-        # double-scaled: near-uniform weights, lse ~ log(i+1) + (small)
+        # double-scaled: logits ~ N(0, 1/96), so over n >= 256 kept keys the
+        # weights are near-uniform and lse ~ log(n) + (a few thousandths)
         i = torch.arange(2048, device=DEV, dtype=torch.float32)
-        gap = (lse[0] - torch.log(i + 1)).abs()
-        assert gap[:, 1:].max().item() < 0.05
+        gap = lse[0] - torch.log(i + 1)
+        assert gap[:, 255:].abs().max().item() < 0.05
+        assert 0.0 < gap[:, 255:].mean().item() < 0.02
 
 
 def test_full_fp16_varlen_sampled():
