@@ -356,7 +356,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (ok && ptx::mbar_wait(&bars->o[sub], 0, kTimeoutNs, &bars->abort)) {
       ptx::tc_fence_after();
       const bool row_ok = r < Lq;
-      const bool empty_row = !(m_run > -INFINITY);
+      // No kept key: l = 0 (O = 0, lse = -inf).  A NaN score leaves l NaN,
+      // which makes both O and lse NaN.
+      const bool empty_row = (l_run == 0.f);
       const float inv = empty_row ? 0.f : 1.f / l_run;
       T* op = static_cast<T*>(p.o) + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)(seq0 + r) * p.os[2];
 #pragma unroll
