@@ -149,6 +149,40 @@ int sdpa_last_launch_count(void);
  */
 int sdpa_take_device_error(int* code);
 
+/* Size of the fixed device scratch array of sdpa_decode_fwd_noalloc(). */
+#define SDPA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * Decode attention that allocates nothing and takes no workspace.  (No
+ * counterpart on the pages: it exists for callers, not for the method.)
+ *
+ * For callers that cannot allocate device memory when they call (a runtime
+ * that reserves all its device memory up front, or a plugin interface that
+ * passes only inputs and outputs): the same split-S decode and combine
+ * kernels as sdpa_fwd(), with their scratch in a 32 MiB array compiled into
+ * the library (SDPA_NOALLOC_SCRATCH_BYTES).  That array occupies 32 MiB on
+ * every GPU where the library's code is loaded, until the process exits.
+ *
+ * Arguments are sdpa_fwd()'s without mask, bias or workspace (mask_kind
+ * NONE).  Takes only problems the decode kernel takes: fp16/bf16,
+ * E = Ev in {64, 128, 256}, (Hq/Hkv)*L <= 8, 16-byte aligned rows; returns
+ * SDPA_ERR_UNSUPPORTED otherwise, and SDPA_ERR_WORKSPACE when the problem
+ * needs more scratch than SDPA_NOALLOC_SCRATCH_BYTES (the same bytes
+ * sdpa_fwd_workspace_size() reports for it).
+ *
+ * The first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress, with that device current; make that first call
+ * before any stream capture.  Every call uses the same array, so calls whose
+ * kernels can overlap on the GPU (other streams, other host threads) race
+ * and must be serialised by the caller.  Nothing in the array needs to be
+ * cleared between calls.
+ */
+int sdpa_decode_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int B, int Hq, int Hkv, int L, int S, int E, int Ev,
+                            const int64_t q_stride[4], const int64_t k_stride[4],
+                            const int64_t v_stride[4], const int64_t o_stride[4],
+                            int has_scale, float scale, int dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

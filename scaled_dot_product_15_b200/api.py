@@ -53,6 +53,11 @@ _SIGNATURES = {
     ),
     "sdpa_last_launch_count": (ctypes.c_int, []),
     "sdpa_take_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
+    "sdpa_decode_fwd_noalloc": (
+        ctypes.c_int,
+        [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 + [_I64x4] * 4
+        + [ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p],
+    ),
 }
 
 _lib = None
