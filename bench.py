@@ -455,6 +455,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=2.0, help="oracle seconds per reference step")
+    ap.add_argument("--bare", action="store_true",
+                    help="only run the workload's launches (for profilers); prints no bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -472,6 +474,12 @@ def main():
     load_library()
     peaks, peak_src = load_peaks()
     w = W.WORKLOADS[args.workload]
+    if args.bare:
+        sets, _ = make_sets(w, device)
+        calls = prepared_calls(w, sets, device)
+        total_ms, kernel_ms, launches = time_device(calls, args.steps, args.warmup, dist_on)
+        print(json.dumps({"bare": w.name, "ms_per_step": total_ms / args.steps, "launches": launches}))
+        return
     sampler = ClockSampler(local)
     res, total_ms, kernel_ms, launches = measure_workload(w, args.steps, args.warmup, peaks, peak_src, device,
                                                          dist_on, sampler)

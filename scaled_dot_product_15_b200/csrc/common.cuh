@@ -7,7 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/sdpa15.h"
+#include "sdpa15.h"
 
 namespace sdpa15 {
 

@@ -10,7 +10,7 @@
 // kept in fp32, and the output accumulator is rescaled by 2^(m_old - m_new)
 // when the maximum grows.
 //
-// B200 mapping (one CTA per 256 query rows of one head; 10 warps):
+// B200 mapping (one CTA per 256 query rows of one head; 12 warps):
 //   warp 9      TMA producer: Q (two 128-row sub-tiles) once, then K_j and V_j
 //               128-key tiles through a ring of shared-memory slots (128-byte
 //               swizzle, 64-column boxes).
@@ -37,6 +37,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
 
 namespace sdpa15 {
@@ -48,9 +49,14 @@ namespace pf {
 constexpr int BM = 128;  // query rows per sub-tile (tensor-memory lanes)
 constexpr int BN = 128;  // keys per tile
 constexpr int NSUB = 2;  // sub-tiles per CTA
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // 3 warpgroups
 constexpr int kWarpMma = 8;
 constexpr int kWarpLoad = 9;
+// Registers: launched with 168 per thread (384 x 168 = 64512); warpgroup 2
+// (MMA, load and two idle warps) drops to 72 so the two softmax warpgroups
+// can rise to 216: 2 x 128 x 216 + 128 x 72 = 64512.
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsOther = 72;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -126,12 +132,72 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t kv_base, int su
   }
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Row maximum of 128 scores held as 4 x 32 raw registers (4 independent
+// chains of three-input max).
+__device__ __forceinline__ float row_max128(const uint32_t (&s)[4][32]) {
+  float a = -INFINITY, b = -INFINITY, c = -INFINITY, d = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      a = fmax3(a, __uint_as_float(s[k][i]), __uint_as_float(s[k][i + 1]));
+      b = fmax3(b, __uint_as_float(s[k][i + 2]), __uint_as_float(s[k][i + 3]));
+      c = fmax3(c, __uint_as_float(s[k][i + 4]), __uint_as_float(s[k][i + 5]));
+      d = fmax3(d, __uint_as_float(s[k][i + 6]), __uint_as_float(s[k][i + 7]));
+    }
+  return fmax3(a, b, fmaxf(c, d));
+}
+
+// P = 2^(S * scale*log2(e) - m) for 128 scores, two at a time (packed fp32
+// FMA), packed to 16-bit pairs in place over the scores (lower key in the low
+// half) and stored over S in tensor memory; returns the row sum of the fp32
+// weights.  With kEmu, 3 of every 8 pairs take the FMA-pipe 2^x so the
+// multi-function unit is not the bottleneck; masked tiles (-inf scores) use
+// the multi-function unit only, whose 2^-inf is exactly 0.
+template <typename T, bool kEmu>
+__device__ __forceinline__ float exp_pack_store(uint32_t (&s)[4][32], float sl, float neg_m, uint32_t tS) {
+  using namespace exp2poly;
+  const uint64_t sl2 = pk(sl, sl), nm2 = pk(neg_m, neg_m);
+  uint64_t acc0 = pk(0.f, 0.f), acc1 = pk(0.f, 0.f);
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int e = 64 * hh + 2 * i;
+      const uint64_t x = ffma2(pk(__uint_as_float(s[e >> 5][e & 31]), __uint_as_float(s[(e + 1) >> 5][(e + 1) & 31])),
+                               sl2, nm2);
+      float x0, x1, p0, p1;
+      upk(x, x0, x1);
+      if (kEmu && (i % 8) < 3) {
+        exp2_pair(x0, x1, p0, p1);
+      } else {
+        p0 = ptx::ex2(x0);
+        p1 = ptx::ex2(x1);
+      }
+      if (i & 1) acc1 = fadd2(acc1, pk(p0, p1));
+      else acc0 = fadd2(acc0, pk(p0, p1));
+      s[2 * hh][i] = pack2<T>(p0, p1);  // s[2hh][>= i] and s[2hh+1] are read first
+    }
+    ptx::tmem_st32(tS + 32 * hh, s[2 * hh]);
+  }
+  float a, b, c, d;
+  upk(acc0, a, b);
+  upk(acc1, c, d);
+  return (a + b) + (c + d);
+}
+
 }  // namespace pf
 
 template <typename T, int D, bool kVarlen>
 __global__ void __launch_bounds__(pf::kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const Params p) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const Params p) {
   using C = pf::Cfg<D>;
   using namespace pf;
   extern __shared__ uint8_t smem_raw[];
@@ -140,19 +206,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* sKV = smem + C::KV_OFF;
   Bars* bars = reinterpret_cast<Bars*>(smem + C::BAR_OFF);
 
-  // ---- work unit: 256 query rows of one (batch, head), or of one segment
-  const int mb = gridDim.x - 1 - blockIdx.x;  // late rows (most keys when causal) first
-  const int h = blockIdx.y;
+  // ---- work unit: 256 query rows of one (batch, head), or of one segment.
+  // Blocks are dispatched in linear order (x fastest), so putting the row
+  // block in z, last rows first, hands out the units with the most key tiles
+  // (causal) first across all heads: greedy longest-first scheduling.
+  const int mb = gridDim.z - 1 - blockIdx.z;
+  const int h = blockIdx.x;
   int b, seq0, Lq, Sk;
   if (kVarlen) {
-    const int sg = blockIdx.z;
+    const int sg = blockIdx.y;
     const int c0 = min(max(__ldg(p.cu + sg), 0), p.L);
     const int c1 = min(max(__ldg(p.cu + sg + 1), c0), p.L);
     b = 0;
     seq0 = c0;
     Lq = Sk = c1 - c0;
   } else {
-    b = blockIdx.z;
+    b = blockIdx.y;
     seq0 = 0;
     Lq = p.L;
     Sk = p.S;
@@ -187,13 +256,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ptx::prefetch_tmap(&tmQ);
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
+    ptx::prefetch_tmap(&tmO);
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem;
-
-  if (warp == kWarpLoad) {
+  if (warp >= 8) {
+   // Warpgroup 2: every warp releases registers at the same instruction, then
+   // splits by role.
+   ptx::regs_dec<kRegsOther>();
+   if (warp == kWarpLoad) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       ptx::mbar_arrive_expect_tx(&bars->q, NSUB * C::TILE);
@@ -231,6 +304,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t idesc_pv = ptx::idesc_f16(kBf16, BM, D, true);
       const uint32_t q_base = ptx::smem_u32(sQ);
       const uint32_t kv_base = ptx::smem_u32(sKV);
+      bool o_done[NSUB] = {false, false};
       bool ok = ptx::mbar_wait(&bars->q, 0, kTimeoutNs, &bars->abort) && ptx::mbar_wait(&bars->full[0], 0, kTimeoutNs, &bars->abort);
       if (ok) {
         ptx::tc_fence_after();
@@ -248,6 +322,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (!ptx::mbar_wait(&bars->p[sub], j & 1, kTimeoutNs, &bars->abort)) { ok = false; break; }
           ptx::tc_fence_after();
           issue_pv<D>(tmem, kv_base, sub, vslot, j > 0, idesc_pv);
+          if (j + 1 == n_kv) {
+            ptx::mma_commit(&bars->o[sub]);  // this sub-tile's output is final
+            o_done[sub] = true;
+          }
           if (j + 1 < n_kv) {
             if (sub == 0) {
               const int kt = 2 * (j + 1);
@@ -264,12 +342,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (kslot >= 0) ptx::mma_commit(&bars->empty[kslot]);
       }
       if (!ok) flag_error(bars, 3);
-      // Completes when every MMA issued above has finished.
-      ptx::mma_commit(&bars->o[0]);
-      ptx::mma_commit(&bars->o[1]);
+      // On an abort, still complete the output barriers once every MMA issued
+      // above has finished, so no waiter is left behind.
+      for (int sub = 0; sub < NSUB; ++sub)
+        if (!o_done[sub]) ptx::mma_commit(&bars->o[sub]);
       if (!ptx::mbar_wait(&bars->o[0], 0, kTimeoutNs, &bars->abort)) flag_error(bars, 4);
     }
+   }
   } else {
+    ptx::regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
     const int sub = warp >> 2;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -291,7 +372,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, s[c]);
       ptx::tmem_wait_ld();
       const int kv0 = j * BN;
-      if (kv0 + BN > Sk || (causal && kv0 + BN - 1 > row_lo)) {
+      const bool masked = kv0 + BN > Sk || (causal && kv0 + BN - 1 > row_lo);  // warp-uniform
+      if (masked) {
         const int lim = causal ? min(Sk, r + 1) : Sk;  // keys [0, lim) are kept
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -299,17 +381,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int i = 0; i < 32; ++i)
             if (kv0 + 32 * c + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          mx0 = fmaxf(mx0, __uint_as_float(s[c][i]));
-          mx1 = fmaxf(mx1, __uint_as_float(s[c][i + 1]));
-          mx2 = fmaxf(mx2, __uint_as_float(s[c][i + 2]));
-          mx3 = fmaxf(mx3, __uint_as_float(s[c][i + 3]));
-        }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl;
+      const float m_tile = row_max128(s) * sl;
       const float m_new = fmaxf(m_run, m_tile);
       const bool need = m_new > m_run + kRescaleLog2;  // false while both are -inf
       const bool any_need = __any_sync(0xffffffffu, need);
@@ -318,23 +390,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         l_run *= factor;
         m_run = m_new;
       }
-      // P = 2^(S*scale*log2e - m), packed two per column in place over the
-      // scores (16-bit pairs, lower key in the low half) and stored over S.
       const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-      float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int e = 64 * hh + 2 * i;
-          const float p0 = ptx::ex2(fmaf(__uint_as_float(s[e >> 5][e & 31]), sl, neg_m));
-          const float p1 = ptx::ex2(fmaf(__uint_as_float(s[(e + 1) >> 5][(e + 1) & 31]), sl, neg_m));
-          rs0 += p0;
-          rs1 += p1;
-          s[2 * hh][i] = pack2<T>(p0, p1);  // reads of s[2hh][>= i] and s[2hh+1] come first
-        }
-        ptx::tmem_st32(tS + 32 * hh, s[2 * hh]);
-      }
+      const float rs = masked ? exp_pack_store<T, false>(s, sl, neg_m, tS) : exp_pack_store<T, true>(s, sl, neg_m, tS);
       // Output rescale (rare): only when some row's maximum grew by > 2^8.
       if (any_need && j > 0) {
 #pragma unroll
@@ -347,7 +404,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           ptx::tmem_st32(tO + 32 * c, o);
         }
       }
-      l_run += rs0 + rs1;
+      l_run += rs;
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars->p[sub]);
@@ -360,20 +417,54 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // which makes both O and lse NaN.
       const bool empty_row = (l_run == 0.f);
       const float inv = empty_row ? 0.f : 1.f / l_run;
-      T* op = static_cast<T*>(p.o) + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)(seq0 + r) * p.os[2];
+      // Rows of this sub-tile that lie in its own sequence can go out through
+      // shared memory and one TMA tensor store (rows past the tensor's end
+      // are clipped by the TMA); a packed sequence's last, partial tile is
+      // written row by row so the next segment's rows are not touched.
+      if (!kVarlen || row_lo + BM <= Lq) {
+        uint8_t* so = sQ + sub * C::TILE;  // this sub-tile's Q tile: its last MMA has completed
+        const uint32_t so_u = ptx::smem_u32(so);
+        const int rin = (warp & 3) * 32 + lane;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        ptx::tmem_ld32(tO + 32 * c, o);
-        ptx::tmem_wait_ld();
-        if (row_ok) {
-          uint32_t w[16];
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tO + 32 * c, o);
+          ptx::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            w[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(op + 32 * c);
+          for (int v = 0; v < 4; ++v) {
+            uint32_t w[4];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+            for (int i = 0; i < 4; ++i)
+              w[i] = pack2<T>(__uint_as_float(o[8 * v + 2 * i]) * inv, __uint_as_float(o[8 * v + 2 * i + 1]) * inv);
+            const int ch = 4 * c + v;  // 16-byte chunk of the row
+            const uint32_t addr = so_u + (ch >> 3) * C::BLOCK + rin * 128 + (((ch & 7) ^ (rin & 7)) << 4);
+            ptx::st_shared_v4(addr, w[0], w[1], w[2], w[3]);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::named_barrier(1 + sub, 128);
+        if ((warp & 3) == 0 && lane == 0) {
+          for (int kb = 0; kb < C::NB; ++kb)
+            ptx::tma_store_4d(&tmO, so + kb * C::BLOCK, 64 * kb, seq0 + row_lo, h, b);
+          ptx::bulk_commit_group();
+          ptx::bulk_wait_read_all();
+        }
+      } else {
+        T* op = static_cast<T*>(p.o) + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)(seq0 + r) * p.os[2];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tO + 32 * c, o);
+          ptx::tmem_wait_ld();
+          if (row_ok) {
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            uint4* dst = reinterpret_cast<uint4*>(op + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          }
         }
       }
       if (row_ok) {
@@ -444,8 +535,9 @@ cudaError_t launch_t(const Params& p, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   const int seqq = p.L, seqk = p.S;
   const int Bm = V ? 1 : p.B;
+  CUtensorMap mo;
   if (!make_map(&mq, p.q, bf16, D, seqq, p.Hq, Bm, p.qs) || !make_map(&mk, p.k, bf16, D, seqk, p.Hkv, Bm, p.ks) ||
-      !make_map(&mv, p.v, bf16, D, seqk, p.Hkv, Bm, p.vs))
+      !make_map(&mv, p.v, bf16, D, seqk, p.Hkv, Bm, p.vs) || !make_map(&mo, p.o, bf16, D, seqq, p.Hq, Bm, p.os))
     return cudaErrorInvalidValue;
   auto kern = prefill_kernel<T, D, V>;
   static bool attr_set = false;  // per instantiation
@@ -456,8 +548,8 @@ cudaError_t launch_t(const Params& p, cudaStream_t st) {
   }
   const int rows = V ? p.max_seqlen : p.L;
   const int mblocks = (rows + pf::NSUB * pf::BM - 1) / (pf::NSUB * pf::BM);
-  dim3 grid(mblocks, p.Hq, V ? p.n_seqs : p.B);
-  kern<<<grid, pf::kThreads, C::SMEM, st>>>(mq, mk, mv, p);
+  dim3 grid(p.Hq, V ? p.n_seqs : p.B, mblocks);
+  kern<<<grid, pf::kThreads, C::SMEM, st>>>(mq, mk, mv, mo, p);
   return cudaGetLastError();
 }
 
@@ -487,6 +579,7 @@ bool prefill_supported(const Params& p, int dtype) {
   if (p.mask == SDPA_MASK_FLOAT_BIAS) return false;
   if (!(p.scale > 0.f) || !isfinite(p.scale)) return false;
   if (p.L < 1 || p.S < 1) return false;
+  if ((int64_t)(p.L + 255) / 256 > 65535) return false;  // row blocks go in grid.z
   if ((p.mask == SDPA_MASK_BLOCK_DIAG || p.mask == SDPA_MASK_BLOCK_DIAG_CAUSAL) && p.n_seqs > 65535) return false;
   if (!strides_ok(p.qs) || !strides_ok(p.ks) || !strides_ok(p.vs) || !strides_ok(p.os)) return false;
   if (!aligned16(p.q) || !aligned16(p.k) || !aligned16(p.v) || !aligned16(p.o)) return false;
