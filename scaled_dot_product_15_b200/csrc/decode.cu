@@ -24,7 +24,7 @@ namespace sdpa15 {
 
 constexpr int kDecThreads = 256;
 constexpr int kDecChunkMax = 1024;  // keys per CTA at most
-constexpr int kDecUnroll = 4;       // keys in flight per lane group
+constexpr int kDecUnroll = 8;       // keys in flight per lane group
 
 // Number of key chunks for a decode problem (also sizes the workspace).
 int decode_splits(int B, int Hkv, int S) {
@@ -102,7 +102,7 @@ __device__ __forceinline__ float group_reduce_rows(float (&v)[R], int lane, int&
 }
 
 template <typename T, int E, int R>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, (R <= 4 ? 3 : 2))
 decode_split_kernel(Params p, int nsplit, int chunk) {
   constexpr int G = E / 8;              // lanes per key row (16-byte slices)
   constexpr int KPW = 32 / G;           // keys per warp step
