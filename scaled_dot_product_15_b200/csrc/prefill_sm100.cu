@@ -100,35 +100,27 @@ __device__ __forceinline__ void flag_error(Bars* bars, int code) {
   atomicCAS(&g_prefill_error, 0, code);
 }
 
-// S_sub = Q_sub K^T over the head dimension, 16 elements per instruction.
-// Both operands are K-major 128-byte-swizzled tiles: a K-step of 16 elements
-// advances the start address by 32 bytes inside the swizzle row, and every
-// 64 elements moves to the next [128 rows][64] block.
-template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t q_base, uint32_t kv_base, int sub, int slot,
-                                         uint32_t idesc) {
+// Lean issue: descriptors built once per CTA, operand addresses are the
+// descriptor plus compile-time offsets (address >> 4 in the low 14 bits never
+// carries inside shared memory).
+template <int D, int SUB>
+__device__ __forceinline__ void issue_qk(uint32_t tmem, uint64_t dq, uint64_t dk, uint32_t idesc) {
   using C = Cfg<D>;
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk / 4) * C::BLOCK + (kk % 4) * 32;
-    const uint64_t a = ptx::sdesc_sw128(q_base + sub * C::TILE + off, 16, 1024);
-    const uint64_t bd = ptx::sdesc_sw128(kv_base + slot * C::TILE + off, 16, 1024);
-    ptx::mma_ss(tmem + sub * 128, a, bd, idesc, kk > 0 ? 1u : 0u);
+    const uint64_t a = dq + (uint64_t)((SUB * C::TILE + off) >> 4);
+    const uint64_t bd = dk + (uint64_t)(off >> 4);
+    ptx::mma_ss(tmem + SUB * 128, a, bd, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
-// O_sub (+)= P_sub V over the 128 keys of a tile, 16 keys per instruction.
-// P is read from tensor memory (16 keys = 8 packed columns); V is an
-// MN-major operand: 16 keys are 16 rows (2048 bytes), the 8-row swizzle
-// atoms are 1024 bytes apart and the 64-column blocks one BLOCK apart.
-template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t kv_base, int sub, int slot, bool acc,
-                                         uint32_t idesc) {
-  using C = Cfg<D>;
+template <int D, int SUB>
+__device__ __forceinline__ void issue_pv(uint32_t tmem, uint64_t dv, uint32_t acc0, uint32_t idesc) {
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
-    const uint64_t bd = ptx::sdesc_sw128(kv_base + slot * C::TILE + kk * 16 * 128, C::BLOCK, 1024);
-    ptx::mma_ts(tmem + 256 + sub * 128, tmem + sub * 128 + kk * 8, bd, idesc, (acc || kk > 0) ? 1u : 0u);
+    const uint64_t bd = dv + (uint64_t)((kk * 16 * 128) >> 4);
+    ptx::mma_ts(tmem + 256 + SUB * 128, tmem + SUB * 128 + kk * 8, bd, idesc, kk > 0 ? 1u : acc0);
   }
 }
 
@@ -157,7 +149,7 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[4][32]) {
 // P = 2^(S * scale*log2(e) - m) for 128 scores, two at a time (packed fp32
 // FMA), packed to 16-bit pairs in place over the scores (lower key in the low
 // half) and stored over S in tensor memory; returns the row sum of the fp32
-// weights.  With kEmu, 3 of every 8 pairs take the FMA-pipe 2^x so the
+// weights.  With kEmu, 2 of every 8 pairs take the FMA-pipe 2^x so the
 // multi-function unit is not the bottleneck; masked tiles (-inf scores) use
 // the multi-function unit only, whose 2^-inf is exactly 0.
 template <typename T, bool kEmu>
@@ -174,7 +166,7 @@ __device__ __forceinline__ float exp_pack_store(uint32_t (&s)[4][32], float sl, 
                                sl2, nm2);
       float x0, x1, p0, p1;
       upk(x, x0, x1);
-      if (kEmu && (i % 8) < 3) {
+      if (kEmu && (i % 8) < 2) {
         exp2_pair(x0, x1, p0, p1);
       } else {
         p0 = ptx::ex2(x0);
@@ -302,15 +294,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
       constexpr uint32_t idesc_qk = ptx::idesc_f16(kBf16, BM, BN, false);
       constexpr uint32_t idesc_pv = ptx::idesc_f16(kBf16, BM, D, true);
-      const uint32_t q_base = ptx::smem_u32(sQ);
-      const uint32_t kv_base = ptx::smem_u32(sKV);
+      const uint64_t dq = ptx::sdesc_sw128(ptx::smem_u32(sQ), 16, 1024);
+      const uint64_t dk0 = ptx::sdesc_sw128(ptx::smem_u32(sKV), 16, 1024);
+      const uint64_t dv0 = ptx::sdesc_sw128(ptx::smem_u32(sKV), C::BLOCK, 1024);
+      constexpr uint64_t kSlotStep = C::TILE >> 4;
       bool o_done[NSUB] = {false, false};
       bool ok = ptx::mbar_wait(&bars->q, 0, kTimeoutNs, &bars->abort) && ptx::mbar_wait(&bars->full[0], 0, kTimeoutNs, &bars->abort);
       if (ok) {
         ptx::tc_fence_after();
-        issue_qk<D>(tmem, q_base, kv_base, 0, 0, idesc_qk);
+        issue_qk<D, 0>(tmem, dq, dk0, idesc_qk);
         ptx::mma_commit(&bars->s[0]);
-        issue_qk<D>(tmem, q_base, kv_base, 1, 0, idesc_qk);
+        issue_qk<D, 1>(tmem, dq, dk0, idesc_qk);
         ptx::mma_commit(&bars->s[1]);
         ptx::mma_commit(&bars->empty[0]);
       }
@@ -321,7 +315,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int sub = 0; sub < NSUB; ++sub) {
           if (!ptx::mbar_wait(&bars->p[sub], j & 1, kTimeoutNs, &bars->abort)) { ok = false; break; }
           ptx::tc_fence_after();
-          issue_pv<D>(tmem, kv_base, sub, vslot, j > 0, idesc_pv);
+          if (sub == 0) issue_pv<D, 0>(tmem, dv0 + vslot * kSlotStep, j > 0 ? 1u : 0u, idesc_pv);
+          else issue_pv<D, 1>(tmem, dv0 + vslot * kSlotStep, j > 0 ? 1u : 0u, idesc_pv);
           if (j + 1 == n_kv) {
             ptx::mma_commit(&bars->o[sub]);  // this sub-tile's output is final
             o_done[sub] = true;
@@ -333,7 +328,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               if (!ptx::mbar_wait(&bars->full[kslot], (kt / C::NS) & 1, kTimeoutNs, &bars->abort)) { ok = false; break; }
               ptx::tc_fence_after();
             }
-            issue_qk<D>(tmem, q_base, kv_base, sub, kslot, idesc_qk);
+            if (sub == 0) issue_qk<D, 0>(tmem, dq, dk0 + kslot * kSlotStep, idesc_qk);
+            else issue_qk<D, 1>(tmem, dq, dk0 + kslot * kSlotStep, idesc_qk);
             ptx::mma_commit(&bars->s[sub]);
           }
         }
@@ -362,7 +358,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      if (!ptx::mbar_wait(&bars->s[sub], j & 1, kTimeoutNs, &bars->abort)) {
+      // Every wait's outcome is made warp-uniform, so a timeout can never
+      // leave part of a warp inside a warp-collective tcgen05 instruction.
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s[sub], j & 1, kTimeoutNs, &bars->abort))) {
         ok = false;
         break;
       }
@@ -410,14 +408,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ptx::mbar_arrive(&bars->p[sub]);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && ptx::mbar_wait(&bars->o[sub], 0, kTimeoutNs, &bars->abort)) {
+    {
+      // Warp-uniform: either the whole warp reads its rows of O or none does.
+      const bool ep_ok = __all_sync(0xffffffffu, ok && ptx::mbar_wait(&bars->o[sub], 0, kTimeoutNs, &bars->abort));
+      if (!ep_ok) flag_error(bars, 5);
       ptx::tc_fence_after();
       const bool row_ok = r < Lq;
       // No kept key: l = 0 (O = 0, lse = -inf).  A NaN score leaves l NaN,
       // which makes both O and lse NaN.
       const bool empty_row = (l_run == 0.f);
       const float inv = empty_row ? 0.f : 1.f / l_run;
-      // Rows of this sub-tile that lie in its own sequence can go out through
+      // Rows of this sub-tile that lie in its own sequence go out through
       // shared memory and one TMA tensor store (rows past the tensor's end
       // are clipped by the TMA); a packed sequence's last, partial tile is
       // written row by row so the next segment's rows are not touched.
@@ -425,31 +426,33 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint8_t* so = sQ + sub * C::TILE;  // this sub-tile's Q tile: its last MMA has completed
         const uint32_t so_u = ptx::smem_u32(so);
         const int rin = (warp & 3) * 32 + lane;
+        if (ep_ok) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          ptx::tmem_ld32(tO + 32 * c, o);
-          ptx::tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            ptx::tmem_ld32(tO + 32 * c, o);
+            ptx::tmem_wait_ld();
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t w[4];
+            for (int v = 0; v < 4; ++v) {
+              uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              w[i] = pack2<T>(__uint_as_float(o[8 * v + 2 * i]) * inv, __uint_as_float(o[8 * v + 2 * i + 1]) * inv);
-            const int ch = 4 * c + v;  // 16-byte chunk of the row
-            const uint32_t addr = so_u + (ch >> 3) * C::BLOCK + rin * 128 + (((ch & 7) ^ (rin & 7)) << 4);
-            ptx::st_shared_v4(addr, w[0], w[1], w[2], w[3]);
+              for (int i = 0; i < 4; ++i)
+                w[i] = pack2<T>(__uint_as_float(o[8 * v + 2 * i]) * inv, __uint_as_float(o[8 * v + 2 * i + 1]) * inv);
+              const int ch = 4 * c + v;  // 16-byte chunk of the row
+              const uint32_t addr = so_u + (ch >> 3) * C::BLOCK + rin * 128 + (((ch & 7) ^ (rin & 7)) << 4);
+              ptx::st_shared_v4(addr, w[0], w[1], w[2], w[3]);
+            }
           }
         }
         ptx::fence_proxy_async_smem();
-        ptx::named_barrier(1 + sub, 128);
-        if ((warp & 3) == 0 && lane == 0) {
+        ptx::named_barrier(1 + sub, 128);  // all 128 threads of the warpgroup, always
+        if ((warp & 3) == 0 && lane == 0 && ep_ok && *reinterpret_cast<volatile int*>(&bars->abort) == 0) {
           for (int kb = 0; kb < C::NB; ++kb)
             ptx::tma_store_4d(&tmO, so + kb * C::BLOCK, 64 * kb, seq0 + row_lo, h, b);
           ptx::bulk_commit_group();
           ptx::bulk_wait_read_all();
         }
-      } else {
+      } else if (ep_ok) {
         T* op = static_cast<T*>(p.o) + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)(seq0 + r) * p.os[2];
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -467,12 +470,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
         }
       }
-      if (row_ok) {
+      if (row_ok && ep_ok) {
         const float lse = empty_row ? -INFINITY : (m_run + __log2f(l_run)) * kLn2;
         p.lse[((int64_t)b * p.Hq + h) * p.L + seq0 + r] = lse;
       }
-    } else {
-      flag_error(bars, 5);
     }
   }
 

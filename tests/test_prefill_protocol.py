@@ -15,9 +15,9 @@ model replays each role's sequence of waits, arrivals, MMA issues and commits
 
 Random interleavings are explored for several tile counts.  Besides deadlock
 and aliasing, every tensor-memory buffer and ring slot carries the tag of what
-was last written to it, so a role reading stale or overwritten data (an S
-buffer reused too early, a key tile released before its MMA ran, an output
-rescaled before its last PV executed) fails the check.
+was last written to it, so a role reading stale or overwritten data (scores
+issued over a P that its PV has not read, a key tile released before its MMA
+ran, an output rescaled before the previous PV executed) fails the check.
 
 The role scripts mirror the kernel; a change to the kernel's protocol must be
 made here too.
@@ -46,22 +46,25 @@ class ProtocolError(AssertionError):
 
 
 class Model:
-    def __init__(self, n_sub, ns, rng):
+    """The kernel's protocol: per sub-tile one score buffer S (P is written
+    over it), one output accumulator O; barriers q, full/empty[ns] (ring),
+    s[sub] (S computed), p[sub] (P written, O rescaled), o[sub] (O final)."""
+
+    def __init__(self, n_kv, ns, rng):
         self.rng = rng
-        self.n_sub = list(n_sub)
-        self.n_kv = max(n_sub)
+        self.n_kv = n_kv
         self.ns = ns
         B = Bar
         self.q = B("q", 1)
         self.full = [B(f"full{i}", 1) for i in range(ns)]
         self.empty = [B(f"empty{i}", 1) for i in range(ns)]
-        self.s = [[B(f"s{a}{b}", 1) for b in range(2)] for a in range(2)]
-        self.p = [[B(f"p{a}{b}", 1) for b in range(2)] for a in range(2)]  # one arrival per warpgroup in the model
+        self.s = [B(f"s{a}", 1) for a in range(2)]
+        self.p = [B(f"p{a}", 1) for a in range(2)]  # one arrival per warpgroup in the model
         self.o = [B(f"o{a}", 1) for a in range(2)]
-        self.done_bar = B("done", 1)
         self.slot = [None] * ns           # tag of the tile in each ring slot
-        self.sbuf = [[None, None], [None, None]]  # tag in each S/P tensor-memory buffer
+        self.sbuf = [None, None]          # tag in each S/P tensor-memory buffer
         self.o_applied = [0, 0]           # PVs executed into O[sub]
+        self.s_exec = [0, 0]              # S MMAs executed per sub-tile
         self.pipe = []                    # in-order tensor pipe
         self.tma = []                     # (slot, tag) loads in flight
 
@@ -81,21 +84,19 @@ class Model:
         if kind == "commit":
             op[1].arrive()
         elif kind == "qk":
-            _, sub, buf, slot, j = op
+            _, sub, slot, j = op
             if self.slot[slot] != ("K", j):
                 raise ProtocolError(f"S{sub}({j}) reads slot {slot} holding {self.slot[slot]}")
-            if self.sbuf[sub][buf] is not None and self.sbuf[sub][buf][0] == "P":
-                pj = self.sbuf[sub][buf][1]
-                if self.o_applied[sub] <= pj:
-                    raise ProtocolError(f"S{sub}({j}) overwrites P({pj}) before its PV ran")
-            self.sbuf[sub][buf] = ("S", j)
-            self._s_exec[sub] = max(self._s_exec[sub], j + 1)
+            if self.sbuf[sub] is not None and self.sbuf[sub][0] == "P" and self.o_applied[sub] <= self.sbuf[sub][1]:
+                raise ProtocolError(f"S{sub}({j}) overwrites P({self.sbuf[sub][1]}) before its PV ran")
+            self.sbuf[sub] = ("S", j)
+            self.s_exec[sub] = j + 1
         elif kind == "pv":
-            _, sub, buf, slot, j = op
+            _, sub, slot, j = op
             if self.slot[slot] != ("V", j):
                 raise ProtocolError(f"PV{sub}({j}) reads slot {slot} holding {self.slot[slot]}")
-            if self.sbuf[sub][buf] != ("P", j):
-                raise ProtocolError(f"PV{sub}({j}) reads buffer holding {self.sbuf[sub][buf]}")
+            if self.sbuf[sub] != ("P", j):
+                raise ProtocolError(f"PV{sub}({j}) reads buffer holding {self.sbuf[sub]}")
             if self.o_applied[sub] != j:
                 raise ProtocolError(f"PV{sub}({j}) out of order")
             self.o_applied[sub] = j + 1
@@ -105,7 +106,7 @@ class Model:
         self.slot[slot] = tag
         self.full[slot].arrive()
 
-    # -- roles (generators yielding callables that return True when they could act)
+    # -- roles: generators yielding ("wait", barrier, parity, phase) ----------
     def producer(self):
         self.q.arrive()  # Q lands (modelled as immediate)
         t = 0
@@ -113,94 +114,66 @@ class Model:
             for which in "KV":
                 slot = t % self.ns
                 yield ("wait", self.empty[slot], ((t // self.ns) & 1) ^ 1, t // self.ns - 1)
-                # the slot is free: nothing may still need its old tile
                 old = self.slot[slot]
-                if old is not None:
-                    self.assert_released(old)
+                if old is not None:  # nothing may still need the old tile
+                    kind, oj = old
+                    for sub in range(2):
+                        if kind == "V" and self.o_applied[sub] <= oj:
+                            raise ProtocolError(f"V{oj} slot refilled before PV{sub}({oj}) ran")
+                        if kind == "K" and self.s_exec[sub] <= oj:
+                            raise ProtocolError(f"K{oj} slot refilled before S{sub}({oj}) ran")
                 self.slot[slot] = ("loading",)
                 self.tma.append((slot, (which, j)))
                 t += 1
 
-    def assert_released(self, tag):
-        kind, j = tag
-        for sub in range(2):
-            if j < self.n_sub[sub]:
-                if kind == "V" and self.o_applied[sub] <= j:
-                    raise ProtocolError(f"V{j} slot refilled before PV{sub}({j}) ran")
-                if kind == "K" and self._s_exec[sub] <= j:
-                    raise ProtocolError(f"K{j} slot refilled before S{sub}({j}) ran")
-
     def mma(self):
-        yield ("wait", self.q, 0, 0)
         ns = self.ns
-
-        def qk(sub, buf, slot, j):
-            self.pipe.append(("qk", sub, buf, slot, j))
-
-        for j in range(min(2, self.n_kv)):
-            kt = 2 * j
-            kslot = kt % ns
-            yield ("wait", self.full[kslot], (kt // ns) & 1, kt // ns)
-            for sub in range(2):
-                if j < self.n_sub[sub]:
-                    qk(sub, j & 1, kslot, j)
-                    self.pipe.append(("commit", self.s[sub][j & 1]))
-            self.pipe.append(("commit", self.empty[kslot]))
+        yield ("wait", self.q, 0, 0)
+        yield ("wait", self.full[0], 0, 0)
+        for sub in range(2):
+            self.pipe.append(("qk", sub, 0, 0))
+            self.pipe.append(("commit", self.s[sub]))
+        self.pipe.append(("commit", self.empty[0]))
         for j in range(self.n_kv):
             vt = 2 * j + 1
             vslot = vt % ns
-            kt = 2 * (j + 2)
-            kslot = kt % ns
-            k_ready = False
             yield ("wait", self.full[vslot], (vt // ns) & 1, vt // ns)
+            kslot = None
             for sub in range(2):
-                if j >= self.n_sub[sub]:
-                    continue
-                yield ("wait", self.p[sub][j & 1], (j >> 1) & 1, j >> 1)
-                self.pipe.append(("pv", sub, j & 1, vslot, j))
-                if j + 2 >= self.n_sub[sub]:
+                yield ("wait", self.p[sub], j & 1, j)
+                self.pipe.append(("pv", sub, vslot, j))
+                if j + 1 == self.n_kv:
                     self.pipe.append(("commit", self.o[sub]))
-                if j + 2 < self.n_sub[sub]:
-                    if not k_ready:
+                if j + 1 < self.n_kv:
+                    if sub == 0:
+                        kt = 2 * (j + 1)
+                        kslot = kt % ns
                         yield ("wait", self.full[kslot], (kt // ns) & 1, kt // ns)
-                        k_ready = True
-                    qk(sub, j & 1, kslot, j + 2)
-                    self.pipe.append(("commit", self.s[sub][j & 1]))
+                    self.pipe.append(("qk", sub, kslot, j + 1))
+                    self.pipe.append(("commit", self.s[sub]))
             self.pipe.append(("commit", self.empty[vslot]))
-            if j + 2 < self.n_kv:
-                if not k_ready:
-                    yield ("wait", self.full[kslot], (kt // ns) & 1, kt // ns)
+            if kslot is not None:
                 self.pipe.append(("commit", self.empty[kslot]))
-        self.pipe.append(("commit", self.done_bar))
-        yield ("wait", self.done_bar, 0, 0)
+        yield ("wait", self.o[0], 0, 0)
 
     def softmax(self, sub):
-        n = self.n_sub[sub]
-        for j in range(n):
-            buf = j & 1
-            yield ("wait", self.s[sub][buf], (j >> 1) & 1, j >> 1)
-            if self.sbuf[sub][buf] != ("S", j):
-                raise ProtocolError(f"softmax{sub}({j}) reads {self.sbuf[sub][buf]}")
-            self.sbuf[sub][buf] = ("P", j)
-            rescale = j > 0 and self.rng.random() < 0.3
-            if j > 0 and j + 1 == n:
-                yield ("wait", self.o[sub], 0, 0)
-            elif j > 0 and rescale:
-                yield ("wait", self.s[sub][(j + 1) & 1], ((j + 1) >> 1) & 1, (j + 1) >> 1)
-            if rescale and self.o_applied[sub] != j:
+        for j in range(self.n_kv):
+            yield ("wait", self.s[sub], j & 1, j)
+            if self.sbuf[sub] != ("S", j):
+                raise ProtocolError(f"softmax{sub}({j}) reads {self.sbuf[sub]}")
+            self.sbuf[sub] = ("P", j)
+            if j > 0 and self.rng.random() < 0.3 and self.o_applied[sub] != j:  # rescale O
                 raise ProtocolError(f"softmax{sub}({j}) rescales O with {self.o_applied[sub]} PVs applied")
-            self.p[sub][buf].arrive()
-        if n > 0:
-            yield ("wait", self.o[sub], 1 if n >= 2 else 0, 1 if n >= 2 else 0)
-            if self.o_applied[sub] != n:
-                raise ProtocolError(f"epilogue{sub} reads O with {self.o_applied[sub]} of {n} PVs")
+            self.p[sub].arrive()
+        yield ("wait", self.o[sub], 0, 0)
+        if self.o_applied[sub] != self.n_kv:
+            raise ProtocolError(f"epilogue{sub} reads O with {self.o_applied[sub]} of {self.n_kv} PVs")
 
     def run(self):
-        self._s_exec = [0, 0]
         roles = [self.producer(), self.mma(), self.softmax(0), self.softmax(1)]
         pending = [None] * len(roles)
         alive = [True] * len(roles)
-        for steps in range(200000):
+        for _ in range(200000):
             choices = []
             # Advance every role to its next wait first (advancing may arrive
             # on barriers), then see which waits can pass.
@@ -234,43 +207,51 @@ class Model:
         raise ProtocolError("did not finish")
 
 
-CASES = [
-    (1, 0), (2, 0), (1, 1), (2, 2), (3, 3), (4, 4), (9, 9), (2, 4), (6, 8), (30, 32), (5, 0), (17, 17),
-]
+CASES = [1, 2, 3, 4, 5, 9, 16, 33]
 
 
-@pytest.mark.parametrize("n_sub", CASES)
-@pytest.mark.parametrize("ns", [8, 16])
-def test_protocol_random_interleavings(n_sub, ns):
-    for seed in range(25):
-        Model(n_sub, ns, random.Random(seed * 1000 + n_sub[0] * 37 + n_sub[1])).run()
+@pytest.mark.parametrize("n_kv", CASES)
+@pytest.mark.parametrize("ns", [4, 8])
+def test_protocol_random_interleavings(n_kv, ns):
+    for seed in range(40):
+        Model(n_kv, ns, random.Random(seed * 1000 + n_kv * 37 + ns)).run()
 
 
-def test_model_catches_single_p_barrier_aliasing():
-    """The protocol with ONE P-ready barrier per sub-tile (instead of one per S
-    buffer) lets the softmax finish two tiles before the MMA issuer waits,
-    aliasing the barrier's parity; the model must flag it."""
+def _caught(cls, n_kv=6, ns=4):
+    for seed in range(300):
+        try:
+            cls(n_kv, ns, random.Random(seed)).run()
+        except ProtocolError:
+            return True
+    return False
 
-    class OneP(Model):
-        def __init__(self, *a):
-            super().__init__(*a)
-            shared = [Bar("p0", 1), Bar("p1", 1)]
-            self.p = [[shared[0], shared[0]], [shared[1], shared[1]]]
 
+def test_model_catches_scores_issued_before_the_pv():
+    """Issuing S(j+1) before PV(j) overwrites P(j) (which lives in S's
+    tensor-memory columns) before the PV reads it."""
+
+    class Early(Model):
         def mma(self):
-            seen = {"p0": 0, "p1": 0}
             for item in Model.mma(self):
-                if item[0] == "wait" and item[1].name in seen:
-                    j = seen[item[1].name]
-                    seen[item[1].name] += 1
-                    item = ("wait", item[1], j & 1, j)
+                # after each PV is queued, move a following S of the same
+                # sub-tile in front of it
+                for k in range(len(self.pipe) - 1):
+                    a, b = self.pipe[k], self.pipe[k + 1]
+                    if a[0] == "pv" and b[0] == "qk" and a[1] == b[1]:
+                        self.pipe[k], self.pipe[k + 1] = b, a
                 yield item
 
-    caught = False
-    for seed in range(200):
-        try:
-            OneP((6, 6), 8, random.Random(seed)).run()
-        except ProtocolError:
-            caught = True
-            break
-    assert caught
+    assert _caught(Early)
+
+
+def test_model_catches_parity_off_by_one():
+    """A softmax that waits for S with the wrong parity passes early."""
+
+    class OffByOne(Model):
+        def softmax(self, sub):
+            for item in Model.softmax(self, sub):
+                if item[1] is self.s[sub]:
+                    item = ("wait", item[1], (item[3] + 1) & 1, item[3])
+                yield item
+
+    assert _caught(OffByOne)
