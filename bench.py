@@ -52,30 +52,41 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
-    """Hash of the CUDA sources, to tell whether stored ncu counters still
-    describe the kernels being timed."""
+# The sources each path's kernels are compiled from.
+KERNEL_SOURCES = {
+    "prefill_tcgen05": ["prefill_sm100.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh"],
+    "decode_split": ["decode.cu", "common.cuh"],
+    "simt": ["simt.cu", "common.cuh"],
+}
+
+
+def kernel_source_hash(path: str = None) -> str:
+    """Hash of the CUDA sources of one path (all sources when None), to tell
+    whether stored ncu counters still describe the kernel being timed."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "scaled_dot_product_15_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    names = KERNEL_SOURCES.get(path) if path else None
+    if names is None:
+        names = [n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh"))]
+    for name in sorted(names):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def stored_traffic(workload: str):
-    """DRAM bytes per launch from a committed ncu capture, if the kernels have
-    not changed since it was taken (else None)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+def stored_traffic(workload: str, path: str):
+    """DRAM bytes per launch of the path's dominant kernel from a committed
+    ncu capture (profiles/traffic.json), if that kernel's sources have not
+    changed since it was taken (else None)."""
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
     try:
-        with open(path) as f:
+        with open(tpath) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
     e = d.get(workload)
-    if not e or e.get("kernel_sha") != kernel_source_hash():
+    if not e or e.get("path") != path or e.get("kernel_sha") != kernel_source_hash(path):
         return None
     return e.get("traffic_bytes_per_launch")
 
@@ -301,7 +312,7 @@ def rate(amount, ms, unit):
     return amount / (ms * 1e-3) / 1e12
 
 
-def roofline(w: W.Workload, kernel_ms: float, peaks, peak_src, sustained=False):
+def roofline(w: W.Workload, kernel_ms: float, peaks, peak_src, path: str, sustained=False):
     amount, unit, bound = work_units(w)
     achieved = rate(amount, kernel_ms, unit)
     if bound == "hbm":
@@ -310,7 +321,7 @@ def roofline(w: W.Workload, kernel_ms: float, peaks, peak_src, sustained=False):
         peak = float(peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"])
         # fp16 dense rate equals bf16 on this tensor core; fp32 runs on FMA units
     return {"bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": unit,
-            "frac": round(achieved / peak, 4), "traffic": stored_traffic(w.name),
+            "frac": round(achieved / peak, 4), "traffic": stored_traffic(w.name, path),
             "peak_source": f"of {peak_src}", "algorithmic_per_launch": amount}
 
 
@@ -326,7 +337,7 @@ def measure_workload(w: W.Workload, steps: int, warmup: int, peaks, peak_src, de
         "ms_per_step": round(total_ms / steps, 5),
         "path": calls[0].plan,
         "gpu_launches": launches,
-        "roofline": roofline(w, kernel_ms, peaks, peak_src),
+        "roofline": roofline(w, kernel_ms, peaks, peak_src, calls[0].plan),
         "l2": (f"{len(sets)} rotating input sets of {set_bytes / 1e6:.1f} MB"
                + (" (all sets fit in L2: latency case)" if len(sets) * set_bytes < L2_BYTES else "")),
     }
@@ -457,6 +468,8 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=2.0, help="oracle seconds per reference step")
     ap.add_argument("--bare", action="store_true",
                     help="only run the workload's launches (for profilers); prints no bench line")
+    ap.add_argument("--bare-batch", type=int, default=0,
+                    help="with --bare: use this batch size instead of the workload's (smaller profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -475,6 +488,10 @@ def main():
     peaks, peak_src = load_peaks()
     w = W.WORKLOADS[args.workload]
     if args.bare:
+        if args.bare_batch:
+            import dataclasses
+
+            w = dataclasses.replace(w, B=args.bare_batch)
         sets, _ = make_sets(w, device)
         calls = prepared_calls(w, sets, device)
         total_ms, kernel_ms, launches = time_device(calls, args.steps, args.warmup, dist_on)
@@ -532,7 +549,7 @@ def main():
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": sampler.summary(),
-            "kernel_sha": kernel_source_hash(),
+            "kernel_sha": kernel_source_hash(res["path"]),
             "workloads": extra,
         }
         print(json.dumps(line), flush=True)
