@@ -10,31 +10,46 @@
 // kept in fp32, and the output accumulator is rescaled by 2^(m_old - m_new)
 // when the maximum grows.
 //
-// B200 mapping (one CTA per 256 query rows of one head; 12 warps):
-//   warp 9      TMA producer: Q (two 128-row sub-tiles) once, then K_j and V_j
-//               128-key tiles through a ring of shared-memory slots (128-byte
-//               swizzle, 64-column boxes).
+// B200 mapping: a persistent kernel, one CTA per SM, 12 warps.  A work unit is
+// 256 query rows (two 128-row sub-tiles) of one (batch, head) or segment.
+// Units are listed longest first (last row blocks first under a causal mask)
+// and handed out through a grid-wide atomic counter, so each CTA takes the
+// next unit when it is ready for one: greedy longest-first scheduling.
+//   warp 9      TMA producer: takes the next unit, publishes it to the other
+//               roles through a small ring in shared memory, then loads K_0,
+//               the unit's Q (each sub-tile's buffer as soon as the previous
+//               unit's last scores of that sub-tile have read it), V_0, K_1,
+//               V_1, ... as 128-key tiles through a ring of shared-memory
+//               slots (128-byte swizzle, 64-column boxes).
 //   warp 8      MMA issuer (one thread): S_i = Q_i K_j^T with both operands in
-//               shared memory, and O_i += P_i V_j with P_i read from tensor
-//               memory; fp32 accumulators live in tensor memory
-//               (S0 | S1 | O0 | O1 = 4 x 128 columns).  The two sub-tiles are
-//               interleaved (PV0, QK0 of the next tile, PV1, QK1) so the tensor
-//               core works on one sub-tile while the other's softmax runs.
+//               shared memory, O_i += P_i V_j with P_i read from tensor memory;
+//               fp32 accumulators in tensor memory (S0 | S1 | O0 | O1 = 512
+//               columns).  Sub-tiles interleave (PV0, S0 next, PV1, S1 next) so
+//               the tensor core runs one while the other's softmax runs; a
+//               sub-tile's first scores of the next unit are issued right
+//               after its last PV of the current one.  Descriptors are built
+//               once; each MMA advances them by compile-time offsets, so the
+//               single issuing thread keeps pace with the tensor core.
 //   warps 0-7   softmax, one thread per query row (warpgroup i owns sub-tile
-//               i): tcgen05.ld of its 128 scores, causal / segment / length
-//               masking on boundary tiles only, row maximum, exp2 with
-//               scale*log2(e) folded into one FMA, P packed to 16 bits and
-//               stored back over its own scores in tensor memory.  The output
-//               is rescaled in tensor memory only when the running maximum
-//               grows by more than 2^8 (a stale maximum is exact because the
-//               final normalisation uses the same one).  Epilogue: O / l to
-//               the output dtype, lse = (m + log2 l) * ln 2.
+//               i): tcgen05.ld of its 128 scores, masking on boundary tiles
+//               only, row maximum, exp2 with scale*log2(e) folded into one
+//               packed FMA (2 of every 8 pairs on the FMA pipe), P packed to
+//               16 bits and stored over its own scores.  The output is
+//               rescaled in tensor memory only when a row maximum grows by more
+//               than 2^8 (exact: the final normalisation uses the same
+//               maximum).  At the end of a unit it writes O / l in the output
+//               dtype straight from tensor memory to global memory and
+//               lse = (m + log2 l) * ln 2, while the next unit's first scores
+//               are already being computed.
 // Causal attention visits only key tiles at or left of the diagonal; packed
 // variable-length batches index tiles from each segment's first token.
 //
 // Every wait on an mbarrier is bounded (2 s); on a timeout the kernel records
-// an error code, drains what it issued and returns.
+// an error code, stops its other roles, drains what it issued and returns.
 #include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "exp2_poly.cuh"
@@ -44,19 +59,32 @@ namespace sdpa15 {
 
 __device__ int g_prefill_error = 0;
 
+// Grid-wide work counters of the persistent prefill kernel, one pair per
+// launch slot: units handed out, CTAs finished.  The last CTA of a launch
+// resets its pair, so a slot is ready again for the next launch that uses
+// it; launches take slots round robin, so up to kSchedSlots launches may run
+// concurrently.
+constexpr int kSchedSlots = 256;
+__device__ unsigned int g_unit_next[kSchedSlots];
+__device__ unsigned int g_cta_done[kSchedSlots];
+
 namespace pf {
 
 constexpr int BM = 128;  // query rows per sub-tile (tensor-memory lanes)
 constexpr int BN = 128;  // keys per tile
-constexpr int NSUB = 2;  // sub-tiles per CTA
+constexpr int NSUB = 2;  // sub-tiles per work unit
 constexpr int kThreads = 384;  // 3 warpgroups
 constexpr int kWarpMma = 8;
 constexpr int kWarpLoad = 9;
-// Registers: launched with 168 per thread (384 x 168 = 64512); warpgroup 2
-// (MMA, load and two idle warps) drops to 72 so the two softmax warpgroups
-// can rise to 216: 2 x 128 x 216 + 128 x 72 = 64512.
+// Registers: the block is launched with 168 per thread (the largest multiple
+// of 8 with 384 x 168 <= 65536), 64512 in all, and setmaxnreg.inc can only
+// redistribute those: warpgroup 2 (MMA, load, two idle warps) drops to 72 so
+// the two softmax warpgroups can rise to 216: 2 x 128 x 216 + 128 x 72 =
+// 64512.  A split above the launch total would wait forever.
 constexpr int kRegsSoftmax = 216;
-constexpr int kRegsOther = 72;
+constexpr int kRegsCtl = 72;
+constexpr int kRegsLaunch = (65536 / kThreads) / 8 * 8;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * kRegsLaunch, "register split");
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -68,18 +96,32 @@ struct Cfg {
   static constexpr int NS = (D <= 64) ? 8 : 4;    // key/value ring slots
   static constexpr int KV_OFF = NSUB * TILE;
   static constexpr int BAR_OFF = KV_OFF + NS * TILE;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  static constexpr int SMEM = BAR_OFF + 512 + 1024;
 };
 
+constexpr int kUnitRing = 4;     // published unit indices in flight
+constexpr int kUnitReaders = 9;  // MMA thread + 8 softmax warps
+
 struct Bars {
-  uint64_t q;
+  uint64_t q[2];         // Q of sub-tile i landed (one phase per unit)
+  uint64_t q_free[2];    // the unit's last score MMAs of sub-tile i have read Q
   uint64_t full[8];
   uint64_t empty[8];
-  uint64_t s[2];
-  uint64_t p[2];
-  uint64_t o[2];
+  uint64_t s[2];         // S[sub] computed (one phase per key tile)
+  uint64_t p[2];         // P[sub] written, O rescaled (one phase per key tile)
+  uint64_t o[2];         // O[sub] final for a unit
+  uint64_t unit_full[kUnitRing];   // a unit index published
+  uint64_t unit_empty[kUnitRing];  // every role has read it
+  uint64_t done;                   // every MMA of the CTA completed
+  int unit[kUnitRing];
   uint32_t tmem;
   int abort;
+};
+static_assert(sizeof(Bars) <= 512, "barrier block");
+
+// A work unit: 256 query rows of one (batch or segment, head).
+struct Unit {
+  int h, b, seq0, Lq, Sk, row0, n_kv;
 };
 
 template <typename T>
@@ -95,32 +137,44 @@ __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+
 __device__ __forceinline__ void flag_error(Bars* bars, int code) {
   *reinterpret_cast<volatile int*>(&bars->abort) = 1;
   atomicCAS(&g_prefill_error, 0, code);
 }
 
+__device__ __forceinline__ bool wait(Bars* bars, uint64_t* bar, uint32_t parity) {
+  return ptx::mbar_wait(bar, parity, kTimeoutNs, &bars->abort);
+}
+
+// Wait for this thread's own asynchronous copies or MMAs to finish before the
+// CTA exits: bounded, but not cut short by another role's abort.
+__device__ __forceinline__ bool drain(uint64_t* bar, uint32_t parity) {
+  const int never = 0;
+  return ptx::mbar_wait(bar, parity, kTimeoutNs, &never);
+}
+
 // Lean issue: descriptors built once per CTA, operand addresses are the
 // descriptor plus compile-time offsets (address >> 4 in the low 14 bits never
-// carries inside shared memory).
-template <int D, int SUB>
-__device__ __forceinline__ void issue_qk(uint32_t tmem, uint64_t dq, uint64_t dk, uint32_t idesc) {
-  using C = Cfg<D>;
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * C::BLOCK + (kk % 4) * 32;
-    const uint64_t a = dq + (uint64_t)((SUB * C::TILE + off) >> 4);
-    const uint64_t bd = dk + (uint64_t)(off >> 4);
-    ptx::mma_ss(tmem + SUB * 128, a, bd, idesc, kk > 0 ? 1u : 0u);
+// carries inside shared memory).  S_i = Q_i K^T: A = Q_i (K-major), B = K
+// tile (K-major), D = tensor-memory columns [i*128, i*128+128).
+template <int D, int KK = 0>
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint64_t dq_i, uint64_t dk, uint32_t idesc) {
+  if constexpr (KK < D / 16) {
+    constexpr uint32_t off = ((KK / 4) * Cfg<D>::BLOCK + (KK % 4) * 32) >> 4;
+    ptx::mma_ss_off<off, off>(tmem_s, dq_i, dk, idesc, KK > 0 ? 1u : 0u);
+    issue_qk<D, KK + 1>(tmem_s, dq_i, dk, idesc);
   }
 }
 
-template <int D, int SUB>
-__device__ __forceinline__ void issue_pv(uint32_t tmem, uint64_t dv, uint32_t acc0, uint32_t idesc) {
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk) {
-    const uint64_t bd = dv + (uint64_t)((kk * 16 * 128) >> 4);
-    ptx::mma_ts(tmem + 256 + SUB * 128, tmem + SUB * 128 + kk * 8, bd, idesc, kk > 0 ? 1u : acc0);
+// O_i += P_i V: A = P_i from tensor memory (16-bit, packed over S_i), B = V
+// tile (MN-major).
+template <int KK = 0>
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t dv, uint32_t acc0,
+                                         uint32_t idesc) {
+  if constexpr (KK < BN / 16) {
+    ptx::mma_ts_off<KK * 8, ((KK * 16 * 128) >> 4)>(tmem_o, tmem_p, dv, idesc, KK > 0 ? 1u : acc0);
+    issue_pv<KK + 1>(tmem_o, tmem_p, dv, acc0, idesc);
   }
 }
 
@@ -184,12 +238,96 @@ __device__ __forceinline__ float exp_pack_store(uint32_t (&s)[4][32], float sl, 
   return (a + b) + (c + d);
 }
 
+// Unit `idx` in longest-first order (the row block outermost, last rows
+// first), or false when it holds no rows (a short packed segment).
+template <bool kVarlen>
+__device__ __forceinline__ bool unit_at(const Params& p, int idx, int bx, int mblocks, bool causal, Unit& u) {
+  const int per = bx * p.Hq;
+  const int mb = mblocks - 1 - idx / per;
+  const int rem = idx - (idx / per) * per;
+  u.h = rem % p.Hq;
+  const int g = rem / p.Hq;
+  if (kVarlen) {
+    const int c0 = min(max(__ldg(p.cu + g), 0), p.L);
+    const int c1 = min(max(__ldg(p.cu + g + 1), c0), p.L);
+    u.b = 0;
+    u.seq0 = c0;
+    u.Lq = u.Sk = c1 - c0;
+  } else {
+    u.b = g;
+    u.seq0 = 0;
+    u.Lq = p.L;
+    u.Sk = p.S;
+  }
+  u.row0 = mb * (NSUB * BM);
+  if (u.row0 >= u.Lq || u.Sk <= 0) return false;
+  int n = (u.Sk + BN - 1) / BN;
+  if (causal) n = min(n, (min(u.row0 + NSUB * BM, u.Lq) - 1) / BN + 1);
+  u.n_kv = n;
+  return true;
+}
+
+// The k-th unit of this CTA as published by the producer: its index in the
+// longest-first list, or -1 when there is no more work.
+__device__ __forceinline__ bool read_unit(Bars* bars, int k, int& idx) {
+  const int e = k % kUnitRing;
+  if (!wait(bars, &bars->unit_full[e], (k / kUnitRing) & 1)) return false;
+  idx = *reinterpret_cast<volatile int*>(&bars->unit[e]);
+  return true;
+}
+
+__device__ __forceinline__ bool publish_unit(Bars* bars, int k, int idx) {
+  const int e = k % kUnitRing;
+  if (!wait(bars, &bars->unit_empty[e], ((k / kUnitRing) & 1) ^ 1)) return false;
+  *reinterpret_cast<volatile int*>(&bars->unit[e]) = idx;
+  ptx::mbar_arrive(&bars->unit_full[e]);
+  return true;
+}
+
+// End of a unit for one sub-tile, by its softmax warpgroup: once the last PV
+// has landed, O / l to the output dtype from tensor memory straight to global
+// memory and lse = (m + log2 l) * ln 2.  Returns false on a timeout.
+template <typename T, int D>
+__device__ __forceinline__ bool store_output(const Params& p, Bars* bars, const Unit& u, int sub, int k, int rin,
+                                             uint32_t tO, float m_run, float l_run) {
+  if (!__all_sync(0xffffffffu, wait(bars, &bars->o[sub], k & 1))) return false;
+  ptx::tc_fence_after();
+  const int r = u.row0 + sub * BM + rin;
+  const bool row_ok = r < u.Lq;
+  // No kept key: l = 0 (O = 0, lse = -inf).  A NaN score leaves l NaN, which
+  // makes both O and lse NaN.
+  const bool empty_row = (l_run == 0.f);
+  const float inv = empty_row ? 0.f : 1.f / l_run;
+  T* op = static_cast<T*>(p.o) + (int64_t)u.b * p.os[0] + (int64_t)u.h * p.os[1] + (int64_t)(u.seq0 + r) * p.os[2];
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    ptx::tmem_ld32(tO + 32 * c, o);
+    ptx::tmem_wait_ld();
+    if (row_ok) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = pack2<T>(__uint_as_float(o[8 * v + 2 * i]) * inv, __uint_as_float(o[8 * v + 2 * i + 1]) * inv);
+        *reinterpret_cast<uint4*>(op + 32 * c + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+  if (row_ok) {
+    const float lse = empty_row ? -INFINITY : (m_run + __log2f(l_run)) * kLn2;
+    p.lse[((int64_t)u.b * p.Hq + u.h) * p.L + u.seq0 + r] = lse;
+  }
+  return true;
+}
+
 }  // namespace pf
 
 template <typename T, int D, bool kVarlen>
 __global__ void __launch_bounds__(pf::kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const Params p) {
+               const __grid_constant__ CUtensorMap tmV, const Params p, int n_units, int mblocks, int sched) {
   using C = pf::Cfg<D>;
   using namespace pf;
   extern __shared__ uint8_t smem_raw[];
@@ -198,45 +336,27 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* sKV = smem + C::KV_OFF;
   Bars* bars = reinterpret_cast<Bars*>(smem + C::BAR_OFF);
 
-  // ---- work unit: 256 query rows of one (batch, head), or of one segment.
-  // Blocks are dispatched in linear order (x fastest), so putting the row
-  // block in z, last rows first, hands out the units with the most key tiles
-  // (causal) first across all heads: greedy longest-first scheduling.
-  const int mb = gridDim.z - 1 - blockIdx.z;
-  const int h = blockIdx.x;
-  int b, seq0, Lq, Sk;
-  if (kVarlen) {
-    const int sg = blockIdx.y;
-    const int c0 = min(max(__ldg(p.cu + sg), 0), p.L);
-    const int c1 = min(max(__ldg(p.cu + sg + 1), c0), p.L);
-    b = 0;
-    seq0 = c0;
-    Lq = Sk = c1 - c0;
-  } else {
-    b = blockIdx.y;
-    seq0 = 0;
-    Lq = p.L;
-    Sk = p.S;
-  }
-  const int row0 = mb * (NSUB * BM);
-  if (row0 >= Lq || Sk <= 0) return;  // uniform over the CTA, before any barrier
   const bool causal = (p.mask == SDPA_MASK_CAUSAL) || (p.mask == SDPA_MASK_BLOCK_DIAG_CAUSAL);
-  int n_kv = (Sk + BN - 1) / BN;
-  if (causal) n_kv = min(n_kv, (min(row0 + NSUB * BM, Lq) - 1) / BN + 1);
-  const int kvh = h / p.group;
+  const int bx = kVarlen ? p.n_seqs : p.B;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    ptx::mbar_init(&bars->q, 1);
-    for (int s = 0; s < C::NS; ++s) {
-      ptx::mbar_init(&bars->full[s], 1);
-      ptx::mbar_init(&bars->empty[s], 1);
-    }
     for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&bars->q[s], 1);
+      ptx::mbar_init(&bars->q_free[s], 1);
       ptx::mbar_init(&bars->s[s], 1);
       ptx::mbar_init(&bars->p[s], 128);
       ptx::mbar_init(&bars->o[s], 1);
     }
+    for (int s = 0; s < C::NS; ++s) {
+      ptx::mbar_init(&bars->full[s], 1);
+      ptx::mbar_init(&bars->empty[s], 1);
+    }
+    for (int e = 0; e < kUnitRing; ++e) {
+      ptx::mbar_init(&bars->unit_full[e], 1);
+      ptx::mbar_init(&bars->unit_empty[e], kUnitReaders);
+    }
+    ptx::mbar_init(&bars->done, 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -248,49 +368,76 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ptx::prefetch_tmap(&tmQ);
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
-    ptx::prefetch_tmap(&tmO);
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem;
+
   if (warp >= 8) {
-   // Warpgroup 2: every warp releases registers at the same instruction, then
-   // splits by role.
-   ptx::regs_dec<kRegsOther>();
-   if (warp == kWarpLoad) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      ptx::mbar_arrive_expect_tx(&bars->q, NSUB * C::TILE);
-      for (int sub = 0; sub < NSUB; ++sub)
-        for (int kb = 0; kb < C::NB; ++kb)
-          ptx::tma_load_4d(sQ + sub * C::TILE + kb * C::BLOCK, &tmQ, &bars->q, 64 * kb, seq0 + row0 + sub * BM, h,
-                           b);
-      int t = 0;
+    // Every warp of a warpgroup changes its register count at the same
+    // instruction, then the warpgroup splits by role.
+    ptx::regs_dec<kRegsCtl>();
+    if (warp == kWarpLoad && lane == 0) {
+      // ---------------------------------------------------------- producer
+      // Takes units from the grid-wide counter (longest first, whichever CTA
+      // is ready next: greedy scheduling), publishes each to the other roles,
+      // then loads K_0, the unit's Q (each sub-tile's buffer once the
+      // previous unit's last scores have read it), V_0, K_1, V_1, ...
+      int t = 0, ku = 0;
+      int nq[NSUB] = {0, 0};  // Q loads issued per sub-tile
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        for (int which = 0; which < 2; ++which, ++t) {
-          const int slot = t % C::NS;
-          if (!ptx::mbar_wait(&bars->empty[slot], ((t / C::NS) & 1) ^ 1, kTimeoutNs, &bars->abort)) {
-            flag_error(bars, 1);
-            ok = false;
-            break;
-          }
-          ptx::mbar_arrive_expect_tx(&bars->full[slot], C::TILE);
-          const CUtensorMap* m = which ? &tmV : &tmK;
-          for (int kb = 0; kb < C::NB; ++kb)
-            ptx::tma_load_4d(sKV + slot * C::TILE + kb * C::BLOCK, m, &bars->full[slot], 64 * kb, seq0 + j * BN,
-                             kvh, b);
+      for (;;) {
+        const int idx = (int)atomicAdd(&g_unit_next[sched], 1u);
+        const bool more = idx < n_units;
+        Unit u;
+        if (more && !unit_at<kVarlen>(p, idx, bx, mblocks, causal, u)) continue;
+        if (!publish_unit(bars, ku, more ? idx : -1)) {
+          ok = false;
+          break;
         }
+        ++ku;
+        if (!more) break;
+        const int kvh = u.h / p.group;
+        for (int j = 0; j < u.n_kv && ok; ++j) {
+          for (int which = 0; which < 2; ++which, ++t) {
+            if (j == 0 && which == 1) {
+              for (int sub = 0; sub < NSUB; ++sub) {
+                if (nq[sub] > 0 && !wait(bars, &bars->q_free[sub], (nq[sub] - 1) & 1)) {
+                  ok = false;
+                  break;
+                }
+                ptx::mbar_arrive_expect_tx(&bars->q[sub], C::TILE);
+                for (int kb = 0; kb < C::NB; ++kb)
+                  ptx::tma_load_4d(sQ + sub * C::TILE + kb * C::BLOCK, &tmQ, &bars->q[sub], 64 * kb,
+                                   u.seq0 + u.row0 + sub * BM, u.h, u.b);
+                ++nq[sub];
+              }
+              if (!ok) break;
+            }
+            const int slot = t % C::NS;
+            if (!wait(bars, &bars->empty[slot], ((t / C::NS) & 1) ^ 1)) {
+              ok = false;
+              break;
+            }
+            ptx::mbar_arrive_expect_tx(&bars->full[slot], C::TILE);
+            const CUtensorMap* m = which ? &tmV : &tmK;
+            for (int kb = 0; kb < C::NB; ++kb)
+              ptx::tma_load_4d(sKV + slot * C::TILE + kb * C::BLOCK, m, &bars->full[slot], 64 * kb,
+                               u.seq0 + j * BN, kvh, u.b);
+          }
+        }
+        if (!ok) break;
       }
-      // Drain: the last load issued into each slot has landed before exit.
-      for (int u = max(0, t - C::NS); u < t; ++u)
-        if (!ptx::mbar_wait(&bars->full[u % C::NS], (u / C::NS) & 1, kTimeoutNs, &bars->abort)) flag_error(bars, 2);
-      if (!ptx::mbar_wait(&bars->q, 0, kTimeoutNs, &bars->abort)) flag_error(bars, 2);
-    }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+      if (!ok) flag_error(bars, 1);
+      // Drain: the last load issued into each slot and each Q buffer has
+      // landed before exit.
+      for (int v = max(0, t - C::NS); v < t; ++v)
+        if (!drain(&bars->full[v % C::NS], (v / C::NS) & 1)) flag_error(bars, 2);
+      for (int sub = 0; sub < NSUB; ++sub)
+        if (nq[sub] > 0 && !drain(&bars->q[sub], (nq[sub] - 1) & 1)) flag_error(bars, 2);
+    } else if (warp == kWarpMma && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
       constexpr uint32_t idesc_qk = ptx::idesc_f16(kBf16, BM, BN, false);
       constexpr uint32_t idesc_pv = ptx::idesc_f16(kBf16, BM, D, true);
@@ -298,183 +445,194 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t dk0 = ptx::sdesc_sw128(ptx::smem_u32(sKV), 16, 1024);
       const uint64_t dv0 = ptx::sdesc_sw128(ptx::smem_u32(sKV), C::BLOCK, 1024);
       constexpr uint64_t kSlotStep = C::TILE >> 4;
-      bool o_done[NSUB] = {false, false};
-      bool ok = ptx::mbar_wait(&bars->q, 0, kTimeoutNs, &bars->abort) && ptx::mbar_wait(&bars->full[0], 0, kTimeoutNs, &bars->abort);
-      if (ok) {
-        ptx::tc_fence_after();
-        issue_qk<D, 0>(tmem, dq, dk0, idesc_qk);
-        ptx::mma_commit(&bars->s[0]);
-        issue_qk<D, 1>(tmem, dq, dk0, idesc_qk);
-        ptx::mma_commit(&bars->s[1]);
-        ptx::mma_commit(&bars->empty[0]);
-      }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int vt = 2 * j + 1, vslot = vt % C::NS;
-        if (!ptx::mbar_wait(&bars->full[vslot], (vt / C::NS) & 1, kTimeoutNs, &bars->abort)) { ok = false; break; }
-        int kslot = -1;
-        for (int sub = 0; sub < NSUB; ++sub) {
-          if (!ptx::mbar_wait(&bars->p[sub], j & 1, kTimeoutNs, &bars->abort)) { ok = false; break; }
+      constexpr uint64_t kSubStep = C::TILE >> 4;
+      int t = 0, k = 0;  // ring position of the unit's K_0; units done
+      int tile0 = 0, tile1 = 0;  // key tiles whose P each sub-tile has handed over
+      int idx = -1;
+      bool ok = read_unit(bars, 0, idx);
+      if (ok) ptx::mbar_arrive(&bars->unit_empty[0]);
+      bool have = ok && idx >= 0;
+      Unit u;
+      if (have) {
+        unit_at<kVarlen>(p, idx, bx, mblocks, causal, u);
+        // Scores of the first unit's first key tile.
+        ok = wait(bars, &bars->full[0], 0);
+#pragma unroll 1
+        for (int sub = 0; sub < NSUB && ok; ++sub) {
+          if (!wait(bars, &bars->q[sub], 0)) {
+            ok = false;
+            break;
+          }
           ptx::tc_fence_after();
-          if (sub == 0) issue_pv<D, 0>(tmem, dv0 + vslot * kSlotStep, j > 0 ? 1u : 0u, idesc_pv);
-          else issue_pv<D, 1>(tmem, dv0 + vslot * kSlotStep, j > 0 ? 1u : 0u, idesc_pv);
-          if (j + 1 == n_kv) {
-            ptx::mma_commit(&bars->o[sub]);  // this sub-tile's output is final
-            o_done[sub] = true;
+          issue_qk<D>(tmem + sub * 128, dq + sub * kSubStep, dk0, idesc_qk);
+          ptx::mma_commit(&bars->s[sub]);
+          if (u.n_kv == 1) ptx::mma_commit(&bars->q_free[sub]);
+        }
+        if (ok) ptx::mma_commit(&bars->empty[0]);
+      }
+      while (have && ok) {
+        const int n = u.n_kv;
+        // Steady key tiles j < n-1: PV_i(j) then S_i(j+1), sub-tile by
+        // sub-tile (S_i then holds only P that its PV has consumed).
+        for (int j = 0; j + 1 < n && ok; ++j) {
+          const int vt = t + 2 * j + 1, vslot = vt % C::NS;
+          const int kt = t + 2 * (j + 1), kslot = kt % C::NS;
+          const uint64_t dv = dv0 + vslot * kSlotStep, dk = dk0 + kslot * kSlotStep;
+          const uint32_t acc = j > 0 ? 1u : 0u;
+          // The first PV of a unit overwrites O: its P is written only after
+          // the softmax warpgroup has read the previous unit's O out.
+          ok = wait(bars, &bars->full[vslot], (vt / C::NS) & 1) && wait(bars, &bars->p[0], tile0 & 1);
+          if (!ok) break;
+          ++tile0;
+          ptx::tc_fence_after();
+          issue_pv(tmem + 256, tmem, dv, acc, idesc_pv);
+          if (!wait(bars, &bars->full[kslot], (kt / C::NS) & 1)) {
+            ok = false;
+            break;
           }
-          if (j + 1 < n_kv) {
-            if (sub == 0) {
-              const int kt = 2 * (j + 1);
-              kslot = kt % C::NS;
-              if (!ptx::mbar_wait(&bars->full[kslot], (kt / C::NS) & 1, kTimeoutNs, &bars->abort)) { ok = false; break; }
-              ptx::tc_fence_after();
-            }
-            if (sub == 0) issue_qk<D, 0>(tmem, dq, dk0 + kslot * kSlotStep, idesc_qk);
-            else issue_qk<D, 1>(tmem, dq, dk0 + kslot * kSlotStep, idesc_qk);
-            ptx::mma_commit(&bars->s[sub]);
+          ptx::tc_fence_after();
+          issue_qk<D>(tmem, dq, dk, idesc_qk);
+          ptx::mma_commit(&bars->s[0]);
+          if (j + 2 == n) ptx::mma_commit(&bars->q_free[0]);  // last scores of the unit
+          if (!wait(bars, &bars->p[1], tile1 & 1)) {
+            ok = false;
+            break;
           }
+          ++tile1;
+          ptx::tc_fence_after();
+          issue_pv(tmem + 384, tmem + 128, dv, acc, idesc_pv);
+          issue_qk<D>(tmem + 128, dq + kSubStep, dk, idesc_qk);
+          ptx::mma_commit(&bars->s[1]);
+          if (j + 2 == n) ptx::mma_commit(&bars->q_free[1]);
+          ptx::mma_commit(&bars->empty[vslot]);
+          ptx::mma_commit(&bars->empty[kslot]);
+        }
+        if (!ok) break;
+        // Last key tile: PV_i(n-1), then the next unit's first scores.
+        const int vt = t + 2 * n - 1, vslot = vt % C::NS;
+        const int kt = t + 2 * n, kslot = kt % C::NS;  // the next unit's K_0
+        int nidx = -1;
+        ok = wait(bars, &bars->full[vslot], (vt / C::NS) & 1) && read_unit(bars, k + 1, nidx);
+        if (!ok) break;
+        ptx::mbar_arrive(&bars->unit_empty[(k + 1) % kUnitRing]);
+        Unit nx;
+        const bool nx_have = nidx >= 0;
+        if (nx_have) unit_at<kVarlen>(p, nidx, bx, mblocks, causal, nx);
+#pragma unroll 1
+        for (int sub = 0; sub < NSUB; ++sub) {
+          if (!wait(bars, &bars->p[sub], (sub ? tile1 : tile0) & 1)) {
+            ok = false;
+            break;
+          }
+          if (sub) ++tile1;
+          else ++tile0;
+          ptx::tc_fence_after();
+          issue_pv(tmem + 256 + sub * 128, tmem + sub * 128, dv0 + vslot * kSlotStep, n > 1 ? 1u : 0u, idesc_pv);
+          ptx::mma_commit(&bars->o[sub]);  // this sub-tile's output is final
+          if (!nx_have) continue;
+          if ((sub == 0 && !wait(bars, &bars->full[kslot], (kt / C::NS) & 1)) ||
+              !wait(bars, &bars->q[sub], (k + 1) & 1)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          issue_qk<D>(tmem + sub * 128, dq + sub * kSubStep, dk0 + kslot * kSlotStep, idesc_qk);
+          ptx::mma_commit(&bars->s[sub]);
+          if (nx.n_kv == 1) ptx::mma_commit(&bars->q_free[sub]);  // the next unit's last scores
         }
         if (!ok) break;
         ptx::mma_commit(&bars->empty[vslot]);
-        if (kslot >= 0) ptx::mma_commit(&bars->empty[kslot]);
+        if (!nx_have) break;
+        ptx::mma_commit(&bars->empty[kslot]);
+        t += 2 * n;
+        ++k;
+        u = nx;
       }
       if (!ok) flag_error(bars, 3);
-      // On an abort, still complete the output barriers once every MMA issued
-      // above has finished, so no waiter is left behind.
-      for (int sub = 0; sub < NSUB; ++sub)
-        if (!o_done[sub]) ptx::mma_commit(&bars->o[sub]);
-      if (!ptx::mbar_wait(&bars->o[0], 0, kTimeoutNs, &bars->abort)) flag_error(bars, 4);
+      // Every MMA issued above completes before tensor memory is freed.
+      ptx::mma_commit(&bars->done);
+      if (!drain(&bars->done, 0)) flag_error(bars, 4);
     }
-   }
   } else {
     ptx::regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
     const int sub = warp >> 2;
+    const int rin = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + sub * 128 + lane_off;
     const uint32_t tO = tmem + 256 + sub * 128 + lane_off;
-    const int row_lo = row0 + sub * BM;
-    const int r = row_lo + (warp & 3) * 32 + lane;  // query row within the sequence
-    const float sl = p.scale_log2;                  // > 0 on this path
-    float m_run = -INFINITY, l_run = 0.f;
+    const float sl = p.scale_log2;  // > 0 on this path
+    int tile = 0;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      // Every wait's outcome is made warp-uniform, so a timeout can never
-      // leave part of a warp inside a warp-collective tcgen05 instruction.
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s[sub], j & 1, kTimeoutNs, &bars->abort))) {
-        ok = false;
-        break;
-      }
-      ptx::tc_fence_after();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, s[c]);
-      ptx::tmem_wait_ld();
-      const int kv0 = j * BN;
-      const bool masked = kv0 + BN > Sk || (causal && kv0 + BN - 1 > row_lo);  // warp-uniform
-      if (masked) {
-        const int lim = causal ? min(Sk, r + 1) : Sk;  // keys [0, lim) are kept
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (kv0 + 32 * c + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
-      }
-      const float m_tile = row_max128(s) * sl;
-      const float m_new = fmaxf(m_run, m_tile);
-      const bool need = m_new > m_run + kRescaleLog2;  // false while both are -inf
-      const bool any_need = __any_sync(0xffffffffu, need);
-      const float factor = need ? ptx::ex2(m_run - m_new) : 1.f;
-      if (need) {
-        l_run *= factor;
-        m_run = m_new;
-      }
-      const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-      const float rs = masked ? exp_pack_store<T, false>(s, sl, neg_m, tS) : exp_pack_store<T, true>(s, sl, neg_m, tS);
-      // Output rescale (rare): only when some row's maximum grew by > 2^8.
-      if (any_need && j > 0) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          ptx::tmem_ld32(tO + 32 * c, o);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-          ptx::tmem_st32(tO + 32 * c, o);
+    for (int k = 0; ok; ++k) {
+      int idx = -1;
+      ok = __all_sync(0xffffffffu, read_unit(bars, k, idx));
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bars->unit_empty[k % kUnitRing]);
+      if (idx < 0) break;
+      Unit u;
+      unit_at<kVarlen>(p, idx, bx, mblocks, causal, u);
+      const int row_lo = u.row0 + sub * BM;
+      const int r = row_lo + rin;  // query row within the sequence
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < u.n_kv; ++j, ++tile) {
+        // Every wait's outcome is made warp-uniform, so a timeout can never
+        // leave part of a warp inside a warp-collective tcgen05 instruction.
+        if (!__all_sync(0xffffffffu, wait(bars, &bars->s[sub], tile & 1))) {
+          ok = false;
+          break;
         }
-      }
-      l_run += rs;
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->p[sub]);
-    }
-    // ------------------------------------------------------------ epilogue
-    {
-      // Warp-uniform: either the whole warp reads its rows of O or none does.
-      const bool ep_ok = __all_sync(0xffffffffu, ok && ptx::mbar_wait(&bars->o[sub], 0, kTimeoutNs, &bars->abort));
-      if (!ep_ok) flag_error(bars, 5);
-      ptx::tc_fence_after();
-      const bool row_ok = r < Lq;
-      // No kept key: l = 0 (O = 0, lse = -inf).  A NaN score leaves l NaN,
-      // which makes both O and lse NaN.
-      const bool empty_row = (l_run == 0.f);
-      const float inv = empty_row ? 0.f : 1.f / l_run;
-      // Rows of this sub-tile that lie in its own sequence go out through
-      // shared memory and one TMA tensor store (rows past the tensor's end
-      // are clipped by the TMA); a packed sequence's last, partial tile is
-      // written row by row so the next segment's rows are not touched.
-      if (!kVarlen || row_lo + BM <= Lq) {
-        uint8_t* so = sQ + sub * C::TILE;  // this sub-tile's Q tile: its last MMA has completed
-        const uint32_t so_u = ptx::smem_u32(so);
-        const int rin = (warp & 3) * 32 + lane;
-        if (ep_ok) {
+        ptx::tc_fence_after();
+        uint32_t s[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, s[c]);
+        ptx::tmem_wait_ld();
+        const int kv0 = j * BN;
+        const bool masked = kv0 + BN > u.Sk || (causal && kv0 + BN - 1 > row_lo);  // warp-uniform
+        if (masked) {
+          const int lim = causal ? min(u.Sk, r + 1) : u.Sk;  // keys [0, lim) are kept
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (kv0 + 32 * c + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
+        }
+        const float m_tile = row_max128(s) * sl;
+        const float m_new = fmaxf(m_run, m_tile);
+        const bool need = m_new > m_run + kRescaleLog2;  // false while both are -inf
+        const bool any_need = __any_sync(0xffffffffu, need);
+        const float factor = need ? ptx::ex2(m_run - m_new) : 1.f;
+        if (need) {
+          l_run *= factor;
+          m_run = m_new;
+        }
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        const float rs =
+            masked ? exp_pack_store<T, false>(s, sl, neg_m, tS) : exp_pack_store<T, true>(s, sl, neg_m, tS);
+        // Output rescale (rare): only when some row's maximum grew by more
+        // than 2^8.  The scores of this tile were issued after the previous
+        // PV, so O holds the sum through the previous tile.
+        if (any_need && j > 0) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
             ptx::tmem_ld32(tO + 32 * c, o);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint32_t w[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                w[i] = pack2<T>(__uint_as_float(o[8 * v + 2 * i]) * inv, __uint_as_float(o[8 * v + 2 * i + 1]) * inv);
-              const int ch = 4 * c + v;  // 16-byte chunk of the row
-              const uint32_t addr = so_u + (ch >> 3) * C::BLOCK + rin * 128 + (((ch & 7) ^ (rin & 7)) << 4);
-              ptx::st_shared_v4(addr, w[0], w[1], w[2], w[3]);
-            }
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+            ptx::tmem_st32(tO + 32 * c, o);
           }
         }
-        ptx::fence_proxy_async_smem();
-        ptx::named_barrier(1 + sub, 128);  // all 128 threads of the warpgroup, always
-        if ((warp & 3) == 0 && lane == 0 && ep_ok && *reinterpret_cast<volatile int*>(&bars->abort) == 0) {
-          for (int kb = 0; kb < C::NB; ++kb)
-            ptx::tma_store_4d(&tmO, so + kb * C::BLOCK, 64 * kb, seq0 + row_lo, h, b);
-          ptx::bulk_commit_group();
-          ptx::bulk_wait_read_all();
-        }
-      } else if (ep_ok) {
-        T* op = static_cast<T*>(p.o) + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)(seq0 + r) * p.os[2];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          ptx::tmem_ld32(tO + 32 * c, o);
-          ptx::tmem_wait_ld();
-          if (row_ok) {
-            uint32_t w[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              w[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-            uint4* dst = reinterpret_cast<uint4*>(op + 32 * c);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-          }
-        }
+        l_run += rs;
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->p[sub]);
       }
-      if (row_ok && ep_ok) {
-        const float lse = empty_row ? -INFINITY : (m_run + __log2f(l_run)) * kLn2;
-        p.lse[((int64_t)b * p.Hq + h) * p.L + seq0 + r] = lse;
-      }
+      if (!ok) break;
+      ok = store_output<T, D>(p, bars, u, sub, k, rin, tO, m_run, l_run);
     }
+    if (!ok) flag_error(bars, 6);
   }
 
   ptx::tc_fence_before();
@@ -482,6 +640,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (warp == kWarpMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
+  }
+  if (tid == 0) {
+    // The last CTA to finish re-arms this launch's scheduler slot.
+    __threadfence();
+    if (atomicAdd(&g_cta_done[sched], 1u) == gridDim.x - 1) {
+      atomicExch(&g_unit_next[sched], 0u);
+      atomicExch(&g_cta_done[sched], 0u);
+      __threadfence();
+    }
   }
 }
 
@@ -521,6 +688,21 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, int D, int seq, int H
   return r == CUDA_SUCCESS;
 }
 
+// Scheduler slot of each launch, round robin over every prefill instantiation.
+std::atomic<unsigned> g_launch_seq{0};
+
+// SMs of the current device (one persistent CTA per SM).
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return 148;
+  if (dev >= 0 && dev < 64) cached[dev] = v;
+  return v;
+}
+
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
 
 bool strides_ok(const int64_t* st) {
@@ -534,23 +716,30 @@ cudaError_t launch_t(const Params& p, cudaStream_t st) {
   using C = pf::Cfg<D>;
   const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap mq, mk, mv;
-  const int seqq = p.L, seqk = p.S;
   const int Bm = V ? 1 : p.B;
-  CUtensorMap mo;
-  if (!make_map(&mq, p.q, bf16, D, seqq, p.Hq, Bm, p.qs) || !make_map(&mk, p.k, bf16, D, seqk, p.Hkv, Bm, p.ks) ||
-      !make_map(&mv, p.v, bf16, D, seqk, p.Hkv, Bm, p.vs) || !make_map(&mo, p.o, bf16, D, seqq, p.Hq, Bm, p.os))
+  if (!make_map(&mq, p.q, bf16, D, p.L, p.Hq, Bm, p.qs) || !make_map(&mk, p.k, bf16, D, p.S, p.Hkv, Bm, p.ks) ||
+      !make_map(&mv, p.v, bf16, D, p.S, p.Hkv, Bm, p.vs))
     return cudaErrorInvalidValue;
   auto kern = prefill_kernel<T, D, V>;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
+    // The warpgroups' setmaxnreg requests must fit in what the block is
+    // launched with, or the increase would wait forever.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * pf::kThreads < 2 * 128 * pf::kRegsSoftmax + 128 * pf::kRegsCtl) return cudaErrorInvalidConfiguration;
     attr_set = true;
   }
   const int rows = V ? p.max_seqlen : p.L;
   const int mblocks = (rows + pf::NSUB * pf::BM - 1) / (pf::NSUB * pf::BM);
-  dim3 grid(p.Hq, V ? p.n_seqs : p.B, mblocks);
-  kern<<<grid, pf::kThreads, C::SMEM, st>>>(mq, mk, mv, mo, p);
+  const int64_t n_units = (int64_t)mblocks * (V ? p.n_seqs : p.B) * p.Hq;
+  if (n_units <= 0 || n_units > (int64_t)(INT32_MAX / 2)) return cudaErrorInvalidValue;
+  const int grid = (int)std::min<int64_t>(n_units, sm_count());
+  const int sched = (int)(g_launch_seq.fetch_add(1) % kSchedSlots);
+  kern<<<grid, pf::kThreads, C::SMEM, st>>>(mq, mk, mv, p, (int)n_units, mblocks, sched);
   return cudaGetLastError();
 }
 
@@ -580,8 +769,6 @@ bool prefill_supported(const Params& p, int dtype) {
   if (p.mask == SDPA_MASK_FLOAT_BIAS) return false;
   if (!(p.scale > 0.f) || !isfinite(p.scale)) return false;
   if (p.L < 1 || p.S < 1) return false;
-  if ((int64_t)(p.L + 255) / 256 > 65535) return false;  // row blocks go in grid.z
-  if ((p.mask == SDPA_MASK_BLOCK_DIAG || p.mask == SDPA_MASK_BLOCK_DIAG_CAUSAL) && p.n_seqs > 65535) return false;
   if (!strides_ok(p.qs) || !strides_ok(p.ks) || !strides_ok(p.vs) || !strides_ok(p.os)) return false;
   if (!aligned16(p.q) || !aligned16(p.k) || !aligned16(p.v) || !aligned16(p.o)) return false;
   return true;

@@ -1,9 +1,14 @@
 """CPU model check of the prefill kernel's synchronisation protocol.
 
-csrc/prefill_sm100.cu runs four roles that meet only on mbarriers: a TMA
-producer, a single-thread tcgen05 MMA issuer and two softmax warpgroups.  This
-model replays each role's sequence of waits, arrivals, MMA issues and commits
-(as written in the kernel) against a model of the hardware:
+csrc/prefill_sm100.cu is a persistent kernel whose four roles meet only on
+mbarriers: a TMA producer, a single-thread tcgen05 MMA issuer and two softmax
+warpgroups (one per 128-row sub-tile, each also writing its sub-tile's output
+at the end of a unit).  A CTA works
+through a list of units (256 query rows each) with a per-unit number of key
+tiles; the producer takes the units and publishes them to the other roles
+through a four-entry ring in shared memory.  This model replays each role's
+sequence of waits, arrivals, MMA issues and commits (as written in the kernel)
+against a model of the hardware:
 
 * an mbarrier completes a phase when its arrival count is reached;
   ``try_wait.parity(P)`` succeeds iff the barrier's current phase parity is
@@ -13,11 +18,14 @@ model replays each role's sequence of waits, arrivals, MMA issues and commits
   once every earlier MMA has executed;
 * TMA loads land at arbitrary later times.
 
-Random interleavings are explored for several tile counts.  Besides deadlock
-and aliasing, every tensor-memory buffer and ring slot carries the tag of what
-was last written to it, so a role reading stale or overwritten data (scores
-issued over a P that its PV has not read, a key tile released before its MMA
-ran, an output rescaled before the previous PV executed) fails the check.
+Random interleavings are explored for several unit lists.  Besides deadlock and
+aliasing, every buffer (Q_i, the key/value ring slots, S/P and O in tensor
+memory) carries the tag of what
+was last written to it, so a role reading stale or overwritten data fails the
+check: scores issued over a P that its PV has not read, a ring slot or the Q
+buffer refilled before the MMAs reading it ran, an output rescaled before the
+previous PV executed, the next unit's first PV overwriting an output that has
+not been read out.
 
 The role scripts mirror the kernel; a change to the kernel's protocol must be
 made here too.
@@ -25,8 +33,6 @@ made here too.
 import random
 
 import pytest
-
-BN = 64  # keys per tile
 
 
 class Bar:
@@ -46,27 +52,39 @@ class ProtocolError(AssertionError):
 
 
 class Model:
-    """The kernel's protocol: per sub-tile one score buffer S (P is written
-    over it), one output accumulator O; barriers q, full/empty[ns] (ring),
-    s[sub] (S computed), p[sub] (P written, O rescaled), o[sub] (O final)."""
+    """Barriers: q[sub] (Q_sub landed), q_free[sub] (last score MMAs of a
+    unit for Q_sub ran), full/empty[ns] (ring), s[sub] (S computed), p[sub]
+    (P written, O rescaled), o[sub] (O final), unit_full/unit_empty[4]
+    (unit ring).  The next unit's first PV needs that unit's first P, which
+    the softmax warpgroup writes only after reading O out, so O needs no
+    release barrier.  Warpgroup arrivals (count 128 in
+    the kernel) and the per-warp unit-ring releases are one arrival per role
+    here."""
 
-    def __init__(self, n_kv, ns, rng):
-        self.rng = rng
-        self.n_kv = n_kv
-        self.ns = ns
+    RING = 4
+    READERS = 3  # MMA, softmax 0, softmax 1
+
+    def __init__(self, units, ns, rng):
+        self.units, self.ns, self.rng = units, ns, rng
         B = Bar
-        self.q = B("q", 1)
+        self.q = [B(f"q{a}", 1) for a in range(2)]
+        self.q_free = [B(f"q_free{a}", 1) for a in range(2)]
         self.full = [B(f"full{i}", 1) for i in range(ns)]
         self.empty = [B(f"empty{i}", 1) for i in range(ns)]
         self.s = [B(f"s{a}", 1) for a in range(2)]
-        self.p = [B(f"p{a}", 1) for a in range(2)]  # one arrival per warpgroup in the model
+        self.p = [B(f"p{a}", 1) for a in range(2)]
         self.o = [B(f"o{a}", 1) for a in range(2)]
-        self.slot = [None] * ns           # tag of the tile in each ring slot
-        self.sbuf = [None, None]          # tag in each S/P tensor-memory buffer
-        self.o_applied = [0, 0]           # PVs executed into O[sub]
-        self.s_exec = [0, 0]              # S MMAs executed per sub-tile
-        self.pipe = []                    # in-order tensor pipe
-        self.tma = []                     # (slot, tag) loads in flight
+        self.unit_full = [B(f"unit_full{e}", 1) for e in range(self.RING)]
+        self.unit_empty = [B(f"unit_empty{e}", self.READERS) for e in range(self.RING)]
+        self.unit = [None] * self.RING   # published unit numbers (-1: no more)
+        self.slot = [None] * ns          # tag of the tile in each ring slot
+        self.qbuf = [None, None]         # tag of each Q_sub buffer
+        self.sbuf = [None, None]         # tag in each S/P tensor-memory buffer
+        self.obuf = [None, None]         # (unit, PVs applied) in each O buffer
+        self.o_read = [None, None]       # last unit whose O was read out
+        self.s_exec = [(-1, 0), (-1, 0)]  # last (unit, tile) S MMA executed per sub-tile
+        self.pipe = []                   # in-order tensor pipe
+        self.tma = []                    # (slot, tag) loads in flight
 
     # -- hardware -------------------------------------------------------
     def check_wait(self, bar, parity, phase):
@@ -80,101 +98,182 @@ class Model:
 
     def exec_pipe(self):
         op = self.pipe.pop(0)
-        kind = op[0]
-        if kind == "commit":
+        if op[0] == "commit":
             op[1].arrive()
-        elif kind == "qk":
-            _, sub, slot, j = op
-            if self.slot[slot] != ("K", j):
-                raise ProtocolError(f"S{sub}({j}) reads slot {slot} holding {self.slot[slot]}")
-            if self.sbuf[sub] is not None and self.sbuf[sub][0] == "P" and self.o_applied[sub] <= self.sbuf[sub][1]:
-                raise ProtocolError(f"S{sub}({j}) overwrites P({self.sbuf[sub][1]}) before its PV ran")
-            self.sbuf[sub] = ("S", j)
-            self.s_exec[sub] = j + 1
-        elif kind == "pv":
-            _, sub, slot, j = op
-            if self.slot[slot] != ("V", j):
-                raise ProtocolError(f"PV{sub}({j}) reads slot {slot} holding {self.slot[slot]}")
-            if self.sbuf[sub] != ("P", j):
-                raise ProtocolError(f"PV{sub}({j}) reads buffer holding {self.sbuf[sub]}")
-            if self.o_applied[sub] != j:
-                raise ProtocolError(f"PV{sub}({j}) out of order")
-            self.o_applied[sub] = j + 1
+            return
+        _, sub, slot, k, j = op
+        if op[0] == "qk":
+            if self.qbuf[sub] != ("Q", k):
+                raise ProtocolError(f"S{sub}({k},{j}) reads the Q{sub} buffer holding {self.qbuf[sub]}")
+            if self.slot[slot] != ("K", k, j):
+                raise ProtocolError(f"S{sub}({k},{j}) reads slot {slot} holding {self.slot[slot]}")
+            sb = self.sbuf[sub]
+            if sb is not None and sb[0] == "P":
+                read = self.obuf[sub] is not None and self.obuf[sub][0] == sb[1] and self.obuf[sub][1] > sb[2]
+                if not read:
+                    raise ProtocolError(f"S{sub}({k},{j}) overwrites P{sb[1:]} before its PV ran")
+            if sb is not None and sb[0] == "S":
+                raise ProtocolError(f"S{sub}({k},{j}) overwrites S{sb[1:]} before the softmax read it")
+            self.sbuf[sub] = ("S", k, j)
+            self.s_exec[sub] = (k, j)
+        else:  # pv
+            if self.slot[slot] != ("V", k, j):
+                raise ProtocolError(f"PV{sub}({k},{j}) reads slot {slot} holding {self.slot[slot]}")
+            if self.sbuf[sub] != ("P", k, j):
+                raise ProtocolError(f"PV{sub}({k},{j}) reads a buffer holding {self.sbuf[sub]}")
+            if j == 0:
+                if self.obuf[sub] is not None and self.o_read[sub] != self.obuf[sub][0]:
+                    raise ProtocolError(f"PV{sub}({k},0) overwrites O of unit {self.obuf[sub][0]} before it was read out")
+                self.obuf[sub] = (k, 1)
+            else:
+                if self.obuf[sub] != (k, j):
+                    raise ProtocolError(f"PV{sub}({k},{j}) out of order: O holds {self.obuf[sub]}")
+                self.obuf[sub] = (k, j + 1)
 
-    def land_tma(self, k):
-        slot, tag = self.tma.pop(k)
-        self.slot[slot] = tag
-        self.full[slot].arrive()
+    def land_tma(self, i):
+        slot, tag = self.tma.pop(i)
+        if slot in ("q0", "q1"):
+            sub = int(slot[1])
+            self.qbuf[sub] = tag
+            self.q[sub].arrive()
+        else:
+            self.slot[slot] = tag
+            self.full[slot].arrive()
+
+    # -- unit ring --------------------------------------------------------
+    def read_unit(self, k):
+        e = k % self.RING
+        yield ("wait", self.unit_full[e], (k // self.RING) & 1, k // self.RING)
+        got = self.unit[e]
+        self.unit_empty[e].arrive()
+        return got
 
     # -- roles: generators yielding ("wait", barrier, parity, phase) ----------
     def producer(self):
-        self.q.arrive()  # Q lands (modelled as immediate)
         t = 0
-        for j in range(self.n_kv):
-            for which in "KV":
-                slot = t % self.ns
-                yield ("wait", self.empty[slot], ((t // self.ns) & 1) ^ 1, t // self.ns - 1)
-                old = self.slot[slot]
-                if old is not None:  # nothing may still need the old tile
-                    kind, oj = old
-                    for sub in range(2):
-                        if kind == "V" and self.o_applied[sub] <= oj:
-                            raise ProtocolError(f"V{oj} slot refilled before PV{sub}({oj}) ran")
-                        if kind == "K" and self.s_exec[sub] <= oj:
-                            raise ProtocolError(f"K{oj} slot refilled before S{sub}({oj}) ran")
-                self.slot[slot] = ("loading",)
-                self.tma.append((slot, (which, j)))
-                t += 1
+        nq = [0, 0]
+        units = list(range(len(self.units))) + [-1]
+        for ku, k in enumerate(units):
+            e = ku % self.RING
+            yield ("wait", self.unit_empty[e], ((ku // self.RING) & 1) ^ 1, ku // self.RING - 1)
+            self.unit[e] = k
+            self.unit_full[e].arrive()
+            if k < 0:
+                return
+            n = self.units[k]
+            for j in range(n):
+                for which in "KV":
+                    if j == 0 and which == "V":
+                        for sub in range(2):
+                            if nq[sub] > 0:
+                                yield ("wait", self.q_free[sub], (nq[sub] - 1) & 1, nq[sub] - 1)
+                                if self.s_exec[sub] < (k - 1, self.units[k - 1] - 1):
+                                    raise ProtocolError(f"Q{sub} of unit {k} loaded under pending score MMAs of unit {k - 1}")
+                            self.qbuf[sub] = ("loading",)
+                            self.tma.append((f"q{sub}", ("Q", k)))
+                            nq[sub] += 1
+                    slot = t % self.ns
+                    yield ("wait", self.empty[slot], ((t // self.ns) & 1) ^ 1, t // self.ns - 1)
+                    old = self.slot[slot]
+                    if old is not None:  # nothing may still need the old tile
+                        kind, ok, oj = old
+                        for sub in range(2):
+                            if kind == "K" and self.s_exec[sub] < (ok, oj):
+                                raise ProtocolError(f"K({ok},{oj}) slot refilled before S{sub} read it")
+                            if kind == "V" and (self.obuf[sub] is None or self.obuf[sub] < (ok, oj + 1)):
+                                raise ProtocolError(f"V({ok},{oj}) slot refilled before PV{sub} read it")
+                    self.slot[slot] = ("loading", -1, -1)
+                    self.tma.append((slot, (which, k, j)))
+                    t += 1
 
     def mma(self):
         ns = self.ns
-        yield ("wait", self.q, 0, 0)
+        t, k, tile = 0, 0, [0, 0]
+        cur = yield from self.read_unit(0)
+        if cur < 0:
+            return
         yield ("wait", self.full[0], 0, 0)
         for sub in range(2):
-            self.pipe.append(("qk", sub, 0, 0))
+            yield ("wait", self.q[sub], 0, 0)
+            self.pipe.append(("qk", sub, 0, cur, 0))
             self.pipe.append(("commit", self.s[sub]))
+            if self.units[cur] == 1:
+                self.pipe.append(("commit", self.q_free[sub]))
         self.pipe.append(("commit", self.empty[0]))
-        for j in range(self.n_kv):
-            vt = 2 * j + 1
-            vslot = vt % ns
-            yield ("wait", self.full[vslot], (vt // ns) & 1, vt // ns)
-            kslot = None
-            for sub in range(2):
-                yield ("wait", self.p[sub], j & 1, j)
-                self.pipe.append(("pv", sub, vslot, j))
-                if j + 1 == self.n_kv:
-                    self.pipe.append(("commit", self.o[sub]))
-                if j + 1 < self.n_kv:
+        while True:
+            n = self.units[cur]
+            # steady key tiles: PV_i(j) then S_i(j+1)
+            for j in range(n - 1):
+                vt, kt = t + 2 * j + 1, t + 2 * (j + 1)
+                vslot, kslot = vt % ns, kt % ns
+                yield ("wait", self.full[vslot], (vt // ns) & 1, vt // ns)
+                for sub in range(2):
+                    yield ("wait", self.p[sub], tile[sub] & 1, tile[sub])
+                    tile[sub] += 1
+                    self.pipe.append(("pv", sub, vslot, cur, j))
                     if sub == 0:
-                        kt = 2 * (j + 1)
-                        kslot = kt % ns
                         yield ("wait", self.full[kslot], (kt // ns) & 1, kt // ns)
-                    self.pipe.append(("qk", sub, kslot, j + 1))
+                    self.pipe.append(("qk", sub, kslot, cur, j + 1))
                     self.pipe.append(("commit", self.s[sub]))
-            self.pipe.append(("commit", self.empty[vslot]))
-            if kslot is not None:
+                    if j + 2 == n:
+                        self.pipe.append(("commit", self.q_free[sub]))
+                self.pipe.append(("commit", self.empty[vslot]))
                 self.pipe.append(("commit", self.empty[kslot]))
-        yield ("wait", self.o[0], 0, 0)
+            # last key tile, then the next unit's first scores
+            vt, kt = t + 2 * n - 1, t + 2 * n
+            vslot, kslot = vt % ns, kt % ns
+            yield ("wait", self.full[vslot], (vt // ns) & 1, vt // ns)
+            nxt = yield from self.read_unit(k + 1)
+            for sub in range(2):
+                yield ("wait", self.p[sub], tile[sub] & 1, tile[sub])
+                tile[sub] += 1
+                self.pipe.append(("pv", sub, vslot, cur, n - 1))
+                self.pipe.append(("commit", self.o[sub]))
+                if nxt < 0:
+                    continue
+                if sub == 0:
+                    yield ("wait", self.full[kslot], (kt // ns) & 1, kt // ns)
+                yield ("wait", self.q[sub], (k + 1) & 1, k + 1)
+                self.pipe.append(("qk", sub, kslot, nxt, 0))
+                self.pipe.append(("commit", self.s[sub]))
+                if self.units[nxt] == 1:
+                    self.pipe.append(("commit", self.q_free[sub]))
+            self.pipe.append(("commit", self.empty[vslot]))
+            if nxt < 0:
+                return
+            self.pipe.append(("commit", self.empty[kslot]))
+            t += 2 * n
+            k += 1
+            cur = nxt
 
     def softmax(self, sub):
-        for j in range(self.n_kv):
-            yield ("wait", self.s[sub], j & 1, j)
-            if self.sbuf[sub] != ("S", j):
-                raise ProtocolError(f"softmax{sub}({j}) reads {self.sbuf[sub]}")
-            self.sbuf[sub] = ("P", j)
-            if j > 0 and self.rng.random() < 0.3 and self.o_applied[sub] != j:  # rescale O
-                raise ProtocolError(f"softmax{sub}({j}) rescales O with {self.o_applied[sub]} PVs applied")
-            self.p[sub].arrive()
-        yield ("wait", self.o[sub], 0, 0)
-        if self.o_applied[sub] != self.n_kv:
-            raise ProtocolError(f"epilogue{sub} reads O with {self.o_applied[sub]} of {self.n_kv} PVs")
+        tile, k = 0, 0
+        while True:
+            cur = yield from self.read_unit(k)
+            if cur < 0:
+                return
+            n = self.units[cur]
+            for j in range(n):
+                yield ("wait", self.s[sub], tile & 1, tile)
+                if self.sbuf[sub] != ("S", cur, j):
+                    raise ProtocolError(f"softmax{sub}({cur},{j}) reads {self.sbuf[sub]}")
+                self.sbuf[sub] = ("P", cur, j)
+                if j > 0 and self.rng.random() < 0.3 and self.obuf[sub] != (cur, j):  # rescale O
+                    raise ProtocolError(f"softmax{sub}({cur},{j}) rescales O holding {self.obuf[sub]}")
+                self.p[sub].arrive()
+                tile += 1
+            # the unit's output of this sub-tile
+            yield ("wait", self.o[sub], k & 1, k)
+            if self.obuf[sub] != (cur, n):
+                raise ProtocolError(f"output({cur},{sub}) reads O holding {self.obuf[sub]}")
+            self.o_read[sub] = cur
+            k += 1
 
     def run(self):
         roles = [self.producer(), self.mma(), self.softmax(0), self.softmax(1)]
         pending = [None] * len(roles)
         alive = [True] * len(roles)
-        for _ in range(200000):
-            choices = []
+        for _ in range(400000):
             # Advance every role to its next wait first (advancing may arrive
             # on barriers), then see which waits can pass.
             for i, g in enumerate(roles):
@@ -183,19 +282,16 @@ class Model:
                         pending[i] = next(g)
                     except StopIteration:
                         alive[i] = False
-            for i in range(len(roles)):
-                if alive[i]:
-                    _, bar, parity, phase = pending[i]
-                    if self.check_wait(bar, parity, phase):
-                        choices.append(("role", i))
+            choices = [("role", i) for i in range(len(roles)) if alive[i] and self.check_wait(*pending[i][1:])]
             if self.pipe:
                 choices.append(("pipe", None))
-            for k in range(len(self.tma)):
-                choices.append(("tma", k))
+            choices += [("tma", i) for i in range(len(self.tma))]
             if not choices:
                 if any(alive):
                     stuck = [pending[i][1].name for i in range(len(roles)) if alive[i]]
                     raise ProtocolError(f"deadlock: roles wait on {stuck}")
+                if self.o_read != [len(self.units) - 1] * 2 and self.units:
+                    raise ProtocolError(f"finished with outputs read up to {self.o_read}")
                 return
             kind, arg = self.rng.choice(choices)
             if kind == "role":
@@ -207,20 +303,20 @@ class Model:
         raise ProtocolError("did not finish")
 
 
-CASES = [1, 2, 3, 4, 5, 9, 16, 33]
+UNIT_LISTS = [[1], [2], [3], [5], [16], [33], [1, 1, 1], [3, 1, 2], [5, 5], [1, 4, 2, 6, 1], [16, 8, 2], [2, 2, 2, 2, 2]]
 
 
-@pytest.mark.parametrize("n_kv", CASES)
+@pytest.mark.parametrize("units", UNIT_LISTS, ids=lambda u: "-".join(map(str, u)))
 @pytest.mark.parametrize("ns", [4, 8])
-def test_protocol_random_interleavings(n_kv, ns):
-    for seed in range(40):
-        Model(n_kv, ns, random.Random(seed * 1000 + n_kv * 37 + ns)).run()
+def test_protocol_random_interleavings(units, ns):
+    for seed in range(30):
+        Model(units, ns, random.Random(seed * 1000 + sum(units) * 37 + ns)).run()
 
 
-def _caught(cls, n_kv=6, ns=4):
+def _caught(cls, units=(3, 1, 4, 2), ns=4):
     for seed in range(300):
         try:
-            cls(n_kv, ns, random.Random(seed)).run()
+            cls(list(units), ns, random.Random(seed)).run()
         except ProtocolError:
             return True
     return False
@@ -255,3 +351,45 @@ def test_model_catches_parity_off_by_one():
                 yield item
 
     assert _caught(OffByOne)
+
+
+def test_model_catches_output_read_before_the_last_pv():
+    """Reading O out without waiting for the unit's last PV reads a partial
+    sum."""
+
+    class NoWait(Model):
+        def softmax(self, sub):
+            for item in Model.softmax(self, sub):
+                if item[1] is self.o[sub]:
+                    continue
+                yield item
+
+    assert _caught(NoWait)
+
+
+def test_model_catches_q_released_too_early():
+    """Releasing Q_i right after a unit's first scores (instead of its last)
+    lets the producer load the next unit's Q under pending score MMAs."""
+
+    class EarlyQ(Model):
+        def mma(self):
+            gen = Model.mma(self)
+            item = next(gen)
+            while True:
+                # drop the kernel's q_free commits; release right after each
+                # sub-tile's first scores of a unit instead
+                for sub in range(2):
+                    qf = ("commit", self.q_free[sub])
+                    while qf in self.pipe:
+                        self.pipe.remove(qf)
+                for i, op in enumerate(list(self.pipe)):
+                    if op[0] == "qk" and op[4] == 0 and ("released", op[1], op[3]) not in self.__dict__.setdefault("rel", set()):
+                        self.rel.add(("released", op[1], op[3]))
+                        self.pipe.insert(self.pipe.index(op) + 1, ("commit", self.q_free[op[1]]))
+                try:
+                    item = gen.send((yield item))
+                except StopIteration:
+                    return
+
+    assert _caught(EarlyQ)
+
