@@ -4,3 +4,4 @@ Only tests, the smoke check and the benchmark's CPU-baseline legs may import
 this package; the product path never does.
 """
 from .sdpa_ref import default_scale, sdpa, sdpa_packed  # noqa: F401
+from .sdpa_bwd_ref import attention_weights, sdpa_backward, sdpa_backward_packed  # noqa: F401

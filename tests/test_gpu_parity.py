@@ -125,6 +125,27 @@ def test_prefill_small(case):
     assert_close(out, lse, ro, rl, dt, str(case))
 
 
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("order", ["growing", "shrinking"])
+def test_prefill_row_maximum_moves_across_tiles(dt, causal, order):
+    """Key norms that grow (or shrink) from tile to tile make every row's
+    maximum jump by far more than the 2^8 the kernel lets its running maximum
+    lag: the rescale of O and the recomputation of a tile's weights must both
+    be exact."""
+    B, H, L, S, E = 1, 2, 300, 1024, 64
+    q = _rand((B, H, L, E), 301, torch.float32)
+    k = _rand((B, H, S, E), 302, torch.float32)
+    v = _rand((B, H, S, E), 303, torch.float32)
+    t = torch.arange(S, dtype=torch.float32) // 128
+    gain = 1.0 + 3.2 * (t if order == "growing" else (t.max() - t))
+    k = k * gain[None, None, :, None]
+    q, k, v = q.to(dt), k.to(dt), v.to(dt)
+    out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), is_causal=causal)
+    ro, rl = ref_sdpa(q, k, v, is_causal=causal)
+    assert_close(out, lse, ro, rl, dt, f"{order} causal={causal}")
+
+
 DECODE_CASES = [
     # dtype, B, Hq, Hkv, L, S, E
     (torch.bfloat16, 2, 8, 2, 1, 3000, 128),
