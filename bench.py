@@ -349,6 +349,41 @@ def measure_workload(w: W.Workload, steps: int, warmup: int, peaks, peak_src, de
     return res, total_ms, kernel_ms, launches
 
 
+def measure_backward(w: W.Workload, steps: int, warmup: int, peaks, peak_src, device):
+    """The gradients of a prefill workload (sdpa_backward for a random output
+    gradient, the forward's out and lse given), timed like the forward.
+    Algorithmic work: 2.5x the forward's flops (five matrix products of the
+    forward's size: S, dP, dV, dK, dQ)."""
+    from scaled_dot_product_15_b200 import sdpa, sdpa_backward
+
+    q, k, v = W.make_inputs(w, device)
+    g = W.randn(tuple(q.shape), w.seed + 100, q.dtype).to(device)
+    causal = w.mask == "causal"
+    out, lse = sdpa(q, k, v, is_causal=causal, scale=w.scale)
+
+    def call():
+        sdpa_backward(q, k, v, out, lse, g, is_causal=causal, scale=w.scale)
+        from scaled_dot_product_15_b200 import api
+
+        return api.last_launch_count()
+
+    total_ms, kernel_ms, launches = time_device([call], steps, warmup, False)
+    amount = 2.5 * W.flops(w)
+    achieved = rate(amount, kernel_ms, "TFLOP/s")
+    peak = float(peaks["bf16_tflops"])
+    return {
+        "value": round(rate(amount, total_ms / steps, "TFLOP/s"), 3),
+        "unit": "TFLOP/s",
+        "ms_per_step": round(total_ms / steps, 5),
+        "path": "backward_simt",
+        "gpu_launches": launches,
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "peak_source": f"of {peak_src}",
+                     "algorithmic_per_launch": amount},
+        "note": "gradients (dq, dk, dv) of this workload; general fp32 SIMT kernels, no tensor cores",
+    }
+
+
 # ----------------------------------------------------------------- CPU oracle
 
 
@@ -523,6 +558,11 @@ def main():
                 extra[name] = r
             except Exception as e:  # report, never hide
                 extra[name] = {"error": repr(e)}
+        if w.mask == "causal" and w.L > 1:
+            try:
+                extra[w.name + ":backward"] = measure_backward(w, 5, 2, peaks, peak_src, device)
+            except Exception as e:
+                extra[w.name + ":backward"] = {"error": repr(e)}
     if rank == 0 and ws == 1:
         cpu = cpu_baseline(w, args.cpu_seconds)
 

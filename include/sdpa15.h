@@ -149,6 +149,57 @@ int sdpa_last_launch_count(void);
  */
 int sdpa_take_device_error(int* code);
 
+/*
+ * Bytes of workspace sdpa_bwd() needs (0 for rejected shapes): one float32
+ * per (batch, query head, query row), rounded up to 256 bytes.
+ */
+size_t sdpa_bwd_workspace_size(int B, int Hq, int Hkv, int L, int S, int E, int Ev,
+                               int mask_kind, int dtype);
+
+/*
+ * Gradients of the attention forward (exactref.ai
+ * "scaled_dot_product_attention", section "er.scaled_dot_product_attention.
+ * backward"): for the output gradient `dout`, with P the forward's weights,
+ *   dP = dout V^T,  D_i = sum_j P_ij dP_ij,  dS = P * (dP - D),
+ *   dv = P^T dout,  dq = scale * dS K,  dk = scale * dS^T Q,
+ * with dk and dv summed over the query heads that share a key/value head.
+ *
+ * q, k, v          the forward's inputs, as for sdpa_fwd().
+ * out, lse         the forward's outputs for these inputs (out in the input
+ *                  dtype with o_stride; lse float32 contiguous (B, Hq, L)).
+ *                  P is recomputed as exp(logit - lse); D_i is computed as
+ *                  dout_i . out_i, equal to sum_j P_ij dP_ij.
+ * dout             output gradient, the shape and dtype of out, element
+ *                  strides do_stride[4] (batch, head, seq, feature).
+ * dq, dk, dv       gradients, written (not accumulated) in the input dtype,
+ *                  shapes of q, k, v, element strides dq_stride, dk_stride,
+ *                  dv_stride.  Every element is written exactly once.
+ * B..Ev, strides of q/k/v/out, has_scale/scale, mask_kind, cu_seqlens,
+ * n_seqs, max_seqlen, bias, bias_stride, dtype: as for sdpa_fwd(); the float
+ * bias gets no gradient.
+ * workspace        device memory of at least sdpa_bwd_workspace_size()
+ *                  bytes, 256-byte aligned, owned by the caller.
+ * stream           cudaStream_t to enqueue on; nothing synchronises.
+ *
+ * Feature strides must be 1.  A row with no kept key contributes 0; a NaN
+ * forward row makes the gradients it touches NaN.  Keys a mask removes are
+ * skipped, so a non-finite value stored under a removed key does not reach
+ * the gradients.  Returns SDPA_OK, SDPA_ERR_INVALID (shapes, strides,
+ * pointers), SDPA_ERR_UNSUPPORTED (head sizes outside 1..256, not an sm_100
+ * device), SDPA_ERR_WORKSPACE or SDPA_ERR_CUDA.
+ */
+int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv,
+             int B, int Hq, int Hkv, int L, int S, int E, int Ev,
+             const int64_t q_stride[4], const int64_t k_stride[4],
+             const int64_t v_stride[4], const int64_t o_stride[4],
+             const int64_t do_stride[4], const int64_t dq_stride[4],
+             const int64_t dk_stride[4], const int64_t dv_stride[4],
+             int has_scale, float scale,
+             int mask_kind, const int32_t* cu_seqlens, int n_seqs, int max_seqlen,
+             const float* bias, const int64_t bias_stride[4],
+             int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Size of the fixed device scratch array of sdpa_decode_fwd_noalloc(). */
 #define SDPA_NOALLOC_SCRATCH_BYTES (32u << 20)
 

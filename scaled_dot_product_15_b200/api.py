@@ -51,6 +51,17 @@ _SIGNATURES = {
         ctypes.c_int,
         [ctypes.c_int] * 7 + [_I64x4] * 4 + [ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4,
     ),
+    "sdpa_bwd_workspace_size": (ctypes.c_size_t, [ctypes.c_int] * 9),
+    "sdpa_bwd": (
+        ctypes.c_int,
+        [ctypes.c_void_p] * 9
+        + [ctypes.c_int] * 7
+        + [_I64x4] * 8
+        + [ctypes.c_int, ctypes.c_float]
+        + [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int]
+        + [ctypes.c_void_p, _I64x4]
+        + [ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
+    ),
     "sdpa_last_launch_count": (ctypes.c_int, []),
     "sdpa_take_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
     "sdpa_decode_fwd_noalloc": (
@@ -238,6 +249,119 @@ def sdpa(
         )
     _check(status, "sdpa_fwd")
     return out, lse
+
+
+def sdpa_backward(
+    query: torch.Tensor,
+    key: torch.Tensor,
+    value: torch.Tensor,
+    out: torch.Tensor,
+    lse: torch.Tensor,
+    grad: torch.Tensor,
+    attn_mask: Optional[torch.Tensor] = None,
+    dropout_p: float = 0.0,
+    is_causal: bool = False,
+    scale: Optional[float] = None,
+    enable_gqa: bool = False,
+    *,
+    layout: str = "bhle",
+    cu_seqlens: Optional[torch.Tensor] = None,
+    max_seqlen: Optional[int] = None,
+) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """(grad_query, grad_key, grad_value) for the output gradient ``grad``,
+    given the forward's inputs and its outputs ``out`` and ``lse`` (as sdpa()
+    returned them); the other arguments are sdpa()'s."""
+    if dropout_p != 0.0:
+        raise ValueError("dropout is random and has no reference; dropout_p must be 0")
+    lib = load_library()
+    for t in (query, key, value, out, grad):
+        if t.dim() != 4 or not t.is_cuda:
+            raise ValueError("query, key, value, out and grad must be 4-D CUDA tensors")
+    if not (query.dtype == key.dtype == value.dtype == out.dtype == grad.dtype):
+        raise ValueError("query, key, value, out and grad must share a dtype")
+    if query.dtype not in _DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {query.dtype}")
+    if cu_seqlens is not None and layout == "bhle":
+        layout = "bmhk"
+    B, Hq, L, E = _dims(query, layout)
+    _, Hkv, S, _ = _dims(key, layout)
+    Ev = _dims(value, layout)[3]
+    if Hq != Hkv and not enable_gqa:
+        raise ValueError("query heads differ from key/value heads: pass enable_gqa=True")
+    if tuple(grad.shape) != tuple(out.shape):
+        raise ValueError("grad must have the output's shape")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, L):
+        raise ValueError("lse must be the forward's contiguous float32 (B, Hq, L) logsumexp")
+    if is_causal and attn_mask is not None:
+        raise ValueError("pass either attn_mask or is_causal, not both")
+    dev = query.device
+    dcode = _DTYPE_CODE[query.dtype]
+    mask_kind = MASK_NONE
+    bias_t, bias_str = None, _i64x4((0, 0, 0, 0))
+    cu_ptr, n_seqs, maxlen = None, 0, 0
+    if cu_seqlens is not None:
+        if attn_mask is not None:
+            raise ValueError("attn_mask cannot be combined with cu_seqlens")
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        mask_kind = MASK_BLOCK_DIAG_CAUSAL if is_causal else MASK_BLOCK_DIAG
+        cu_ptr, n_seqs, maxlen = cu_seqlens.data_ptr(), cu_seqlens.numel() - 1, int(max_seqlen)
+    elif is_causal:
+        mask_kind = MASK_CAUSAL
+    elif attn_mask is not None:
+        mask_kind = MASK_FLOAT_BIAS
+        m = attn_mask.to(dev)
+        if m.dtype == torch.bool:
+            m = torch.where(m, 0.0, float("-inf")).to(torch.float32)
+        elif m.dtype != torch.float32:
+            m = m.to(torch.float32)
+        bias_t = m.expand(B, Hq, L, S)
+        bias_str = _i64x4(bias_t.stride())
+    dq, dk, dv = torch.empty_like(query), torch.empty_like(key), torch.empty_like(value)
+    strides = [_i64x4(_strides(t, layout)) for t in (query, key, value, out, grad, dq, dk, dv)]
+    ws_bytes = lib.sdpa_bwd_workspace_size(B, Hq, Hkv, L, S, E, Ev, mask_kind, dcode)
+    ws = _workspace(dev, ws_bytes)
+    ws_ptr = None if ws is None else (ws.data_ptr() + 255) // 256 * 256
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        status = lib.sdpa_bwd(
+            query.data_ptr(), key.data_ptr(), value.data_ptr(), out.data_ptr(), lse.data_ptr(),
+            grad.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+            B, Hq, Hkv, L, S, E, Ev, *strides,
+            0 if scale is None else 1, 0.0 if scale is None else float(scale),
+            mask_kind, cu_ptr, n_seqs, maxlen,
+            None if bias_t is None else bias_t.data_ptr(), bias_str,
+            dcode, ws_ptr, ws_bytes, stream,
+        )
+    _check(status, "sdpa_bwd")
+    return dq, dk, dv
+
+
+class _Attention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, query, key, value, is_causal, scale, enable_gqa, layout, cu_seqlens, max_seqlen):
+        out, lse = sdpa(query, key, value, is_causal=is_causal, scale=scale, enable_gqa=enable_gqa,
+                        layout=layout, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen)
+        ctx.save_for_backward(query, key, value, out, lse)
+        ctx.args = (is_causal, scale, enable_gqa, layout, cu_seqlens, max_seqlen)
+        ctx.mark_non_differentiable(lse)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, grad_out, grad_lse):
+        query, key, value, out, lse = ctx.saved_tensors
+        is_causal, scale, enable_gqa, layout, cu_seqlens, max_seqlen = ctx.args
+        dq, dk, dv = sdpa_backward(query, key, value, out, lse, grad_out.contiguous(), is_causal=is_causal,
+                                   scale=scale, enable_gqa=enable_gqa, layout=layout, cu_seqlens=cu_seqlens,
+                                   max_seqlen=max_seqlen)
+        return dq, dk, dv, None, None, None, None, None, None
+
+
+def attention(query, key, value, is_causal=False, scale=None, enable_gqa=False, *, layout="bhle",
+              cu_seqlens=None, max_seqlen=None) -> torch.Tensor:
+    """sdpa() as a differentiable op: returns the output; its backward runs
+    sdpa_backward() (the logsumexp is kept for it, not differentiated)."""
+    return _Attention.apply(query, key, value, is_causal, scale, enable_gqa, layout, cu_seqlens, max_seqlen)[0]
 
 
 def plan(query, key, value, *, layout="bhle", mask_kind=MASK_NONE, out=None) -> str:

@@ -14,6 +14,8 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int L, int S, int Ev);
 bool prefill_supported(const Params& p, int dtype);
 cudaError_t launch_prefill(const Params& p, int dtype, cudaStream_t st);
 cudaError_t prefill_take_error(int* code);
+cudaError_t launch_backward(const Params& p, const BwdParams& g, int dtype, cudaStream_t st, int* launches);
+size_t backward_workspace_bytes(int B, int Hq, int L);
 }  // namespace sdpa15
 
 using namespace sdpa15;
@@ -180,6 +182,76 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
     err = launch_simt(p, dtype, cs);
   }
   if (err != cudaSuccess) return SDPA_ERR_CUDA;
+  t_last_launches = launches;
+  return SDPA_OK;
+}
+
+size_t sdpa_bwd_workspace_size(int B, int Hq, int Hkv, int L, int S, int E, int Ev, int mask_kind,
+                               int dtype) {
+  const int64_t z[4] = {0, 0, 0, 1};
+  if (check_shapes(B, Hq, Hkv, L, S, E, Ev, z, z, z, z, mask_kind, dtype) != SDPA_OK) return 0;
+  return backward_workspace_bytes(B, Hq, L);
+}
+
+int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int L, int S,
+             int E, int Ev, const int64_t q_stride[4], const int64_t k_stride[4],
+             const int64_t v_stride[4], const int64_t o_stride[4], const int64_t do_stride[4],
+             const int64_t dq_stride[4], const int64_t dk_stride[4], const int64_t dv_stride[4],
+             int has_scale, float scale, int mask_kind, const int32_t* cu_seqlens, int n_seqs,
+             int max_seqlen, const float* bias, const int64_t bias_stride[4], int dtype,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  t_last_launches = 0;
+  int st = check_shapes(B, Hq, Hkv, L, S, E, Ev, q_stride, k_stride, v_stride, o_stride, mask_kind, dtype);
+  if (st != SDPA_OK) return st;
+  // The gradients' strides follow the same rules as the forward's tensors.
+  st = check_shapes(B, Hq, Hkv, L, S, E, Ev, dq_stride, dk_stride, dv_stride, do_stride, mask_kind, dtype);
+  if (st != SDPA_OK) return st;
+  if (has_scale && !isfinite(scale)) return SDPA_ERR_INVALID;
+  if (B == 0) return SDPA_OK;
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return SDPA_ERR_INVALID;
+  if (mask_kind == SDPA_MASK_BLOCK_DIAG || mask_kind == SDPA_MASK_BLOCK_DIAG_CAUSAL) {
+    if (!cu_seqlens || n_seqs < 1 || max_seqlen < 1) return SDPA_ERR_INVALID;
+  }
+  if (mask_kind == SDPA_MASK_FLOAT_BIAS) {
+    if (!bias || !bias_stride) return SDPA_ERR_INVALID;
+    for (int d = 0; d < 4; ++d)
+      if (bias_stride[d] < 0) return SDPA_ERR_INVALID;
+  }
+  const size_t need = backward_workspace_bytes(B, Hq, L);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need ||
+                   reinterpret_cast<uintptr_t>(workspace) % 256 != 0))
+    return SDPA_ERR_WORKSPACE;
+  if (!is_sm100()) return SDPA_ERR_UNSUPPORTED;
+
+  Params p;
+  fill_params(p, q, k, v, const_cast<void*>(out), const_cast<float*>(lse), B, Hq, Hkv, L, S, E, Ev, q_stride,
+              k_stride, v_stride, o_stride, mask_kind);
+  p.scale = has_scale ? scale : (float)(1.0 / sqrt((double)E));
+  p.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
+  p.cu = cu_seqlens;
+  p.n_seqs = n_seqs;
+  p.max_seqlen = max_seqlen;
+  if (mask_kind == SDPA_MASK_FLOAT_BIAS) {
+    p.bias = bias;
+    for (int d = 0; d < 4; ++d) p.bs[d] = bias_stride[d];
+  }
+  BwdParams g;
+  memset(&g, 0, sizeof(g));
+  g.dO = dout;
+  g.dq = dq;
+  g.dk = dk;
+  g.dv = dv;
+  for (int d = 0; d < 4; ++d) {
+    g.dos[d] = do_stride[d];
+    g.dqs[d] = dq_stride[d];
+    g.dks[d] = dk_stride[d];
+    g.dvs[d] = dv_stride[d];
+  }
+  g.D = static_cast<float*>(workspace);
+  int launches = 0;
+  if (launch_backward(p, g, dtype, static_cast<cudaStream_t>(stream), &launches) != cudaSuccess)
+    return SDPA_ERR_CUDA;
   t_last_launches = launches;
   return SDPA_OK;
 }

@@ -107,3 +107,41 @@ def test_dispatch_plan():
     assert _plan(64, 32, 8, 1, 16384, 128, 128, 0, api.SDPA_BF16, align=2) == 3  # unaligned
     assert _plan(1, 2, 2, 64, 64, 48, 48, api.MASK_FLOAT_BIAS, api.SDPA_F16) == 3
     assert _plan(1, 3, 2, 64, 64, 64, 64, 0, api.SDPA_F16) == -api.SDPA_ERR_INVALID
+
+
+def _bwd(**kw):
+    lib = api.load_library()
+    a = dict(B=1, Hq=2, Hkv=2, L=8, S=8, E=64, Ev=64, mask=0, dtype=api.SDPA_BF16, ws=None, ws_bytes=0,
+             scale=None)
+    a.update(kw)
+    fake = 0x10000  # never dereferenced: every case below fails on the host
+    sq = api._i64x4((a["Hq"] * a["L"] * a["E"], a["L"] * a["E"], a["E"], 1))
+    sk = api._i64x4((a["Hkv"] * a["S"] * a["E"], a["S"] * a["E"], a["E"], 1))
+    sv = api._i64x4((a["Hkv"] * a["S"] * a["Ev"], a["S"] * a["Ev"], a["Ev"], 1))
+    so = api._i64x4((a["Hq"] * a["L"] * a["Ev"], a["L"] * a["Ev"], a["Ev"], 1))
+    sdq = api._i64x4(kw.get("dqstride", (a["Hq"] * a["L"] * a["E"], a["L"] * a["E"], a["E"], 1)))
+    ptr = kw.get("ptr", fake)
+    return lib.sdpa_bwd(fake, fake, fake, fake, fake, fake, ptr, fake, fake,
+                        a["B"], a["Hq"], a["Hkv"], a["L"], a["S"], a["E"], a["Ev"],
+                        sq, sk, sv, so, so, sdq, sk, sv, 0 if a["scale"] is None else 1, a["scale"] or 0.0,
+                        a["mask"], None, 0, 0, None, api._i64x4((0, 0, 0, 0)), a["dtype"], a["ws"],
+                        a["ws_bytes"], None)
+
+
+def test_backward_host_side_rejections_and_workspace():
+    lib = api.load_library()
+    assert lib.sdpa_bwd_workspace_size(4, 16, 16, 2048, 2048, 128, 128, api.MASK_CAUSAL, api.SDPA_BF16) == 4 * 16 * 2048 * 4
+    assert lib.sdpa_bwd_workspace_size(1, 3, 2, 8, 8, 64, 64, 0, api.SDPA_BF16) == 0  # invalid shape
+    assert lib.sdpa_bwd_workspace_size(1, 2, 2, 3, 8, 64, 64, 0, api.SDPA_BF16) == 256  # rounded up
+    assert _bwd(Hq=3, Hkv=2) == api.SDPA_ERR_INVALID
+    assert _bwd(E=300) == api.SDPA_ERR_UNSUPPORTED
+    assert _bwd(dqstride=(1, 1, 1, 2)) == api.SDPA_ERR_INVALID     # a gradient's feature stride
+    assert _bwd(scale=float("inf")) == api.SDPA_ERR_INVALID
+    assert _bwd(ptr=None) == api.SDPA_ERR_INVALID                   # missing dq
+    assert _bwd() == api.SDPA_ERR_WORKSPACE                         # D needs workspace
+    import torch
+
+    if not torch.cuda.is_available():  # with a GPU this would launch on fake pointers
+        assert _bwd(ws=0x10100, ws_bytes=256) == api.SDPA_ERR_UNSUPPORTED
+    assert _bwd(ws=0x10180, ws_bytes=256) == api.SDPA_ERR_WORKSPACE  # not 256-byte aligned
+    assert _bwd(B=0) == api.SDPA_OK
