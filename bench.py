@@ -57,6 +57,7 @@ KERNEL_SOURCES = {
     "prefill_tcgen05": ["prefill_sm100.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh"],
     "decode_split": ["decode.cu", "common.cuh"],
     "simt": ["simt.cu", "common.cuh"],
+    "backward_simt": ["backward_simt.cu", "backward.cuh", "common.cuh"],
 }
 
 

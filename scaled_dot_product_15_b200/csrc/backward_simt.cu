@@ -20,7 +20,7 @@
 // forward row (lse NaN) makes what it touches NaN.  Removed keys are skipped,
 // so a non-finite value under a removed key does not reach the gradients
 // (the page's literal rule would make that row's D NaN).
-#include "common.cuh"
+#include "backward.cuh"
 
 namespace sdpa15 {
 

@@ -4,7 +4,7 @@
 #include <math.h>
 #include <string.h>
 
-#include "common.cuh"
+#include "backward.cuh"
 
 namespace sdpa15 {
 cudaError_t launch_simt(const Params& p, int dtype, cudaStream_t st);
