@@ -58,6 +58,8 @@ KERNEL_SOURCES = {
     "decode_split": ["decode.cu", "common.cuh"],
     "simt": ["simt.cu", "common.cuh"],
     "backward_simt": ["backward_simt.cu", "backward.cuh", "common.cuh"],
+    "backward_tcgen05": ["backward_sm100.cu", "backward_simt.cu", "backward.cuh", "tma_host.cuh", "sm100_ptx.cuh",
+                         "common.cuh"],
 }
 
 
@@ -369,6 +371,9 @@ def measure_backward(w: W.Workload, steps: int, warmup: int, peaks, peak_src, de
         return api.last_launch_count()
 
     total_ms, kernel_ms, launches = time_device([call], steps, warmup, False)
+    from scaled_dot_product_15_b200.api import backward_plan
+
+    path = backward_plan(q, k, v, g, mask_kind=1 if causal else 0)
     amount = 2.5 * W.flops(w)
     achieved = rate(amount, kernel_ms, "TFLOP/s")
     peak = float(peaks["bf16_tflops"])
@@ -376,12 +381,12 @@ def measure_backward(w: W.Workload, steps: int, warmup: int, peaks, peak_src, de
         "value": round(rate(amount, total_ms / steps, "TFLOP/s"), 3),
         "unit": "TFLOP/s",
         "ms_per_step": round(total_ms / steps, 5),
-        "path": "backward_simt",
+        "path": path,
         "gpu_launches": launches,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": None, "peak_source": f"of {peak_src}",
                      "algorithmic_per_launch": amount},
-        "note": "gradients (dq, dk, dv) of this workload; general fp32 SIMT kernels, no tensor cores",
+        "note": "gradients (dq, dk, dv) of this workload: row-dot, dK/dV and dQ kernels",
     }
 
 

@@ -184,7 +184,9 @@ size_t sdpa_bwd_workspace_size(int B, int Hq, int Hkv, int L, int S, int E, int 
  * Feature strides must be 1.  A row with no kept key contributes 0; a NaN
  * forward row makes the gradients it touches NaN.  Keys a mask removes are
  * skipped, so a non-finite value stored under a removed key does not reach
- * the gradients.  Returns SDPA_OK, SDPA_ERR_INVALID (shapes, strides,
+ * the gradients.  Kernels: a row-dot kernel for D, then either the tcgen05
+ * dK/dV and dQ kernels (see sdpa_bwd_plan) or the general SIMT ones; each
+ * output element is written once, so results are deterministic.  Returns SDPA_OK, SDPA_ERR_INVALID (shapes, strides,
  * pointers), SDPA_ERR_UNSUPPORTED (head sizes outside 1..256, not an sm_100
  * device), SDPA_ERR_WORKSPACE or SDPA_ERR_CUDA.
  */
@@ -199,6 +201,22 @@ int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const
              int mask_kind, const int32_t* cu_seqlens, int n_seqs, int max_seqlen,
              const float* bias, const int64_t bias_stride[4],
              int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Which kernels sdpa_bwd() would run for these arguments (no work is done):
+ * 1 = the tcgen05/TMA backward (fp16/bf16, E = Ev in {64, 96, 128}, mask
+ * none / causal / block-diagonal, TMA-legal strides and 16-byte aligned
+ * pointers), 3 = the general SIMT kernels, or a negative sdpa_status for
+ * rejected arguments.  The varlen limits (n_seqs, max_seqlen) are not
+ * checked here.
+ */
+int sdpa_bwd_plan(int B, int Hq, int Hkv, int L, int S, int E, int Ev,
+                  const int64_t q_stride[4], const int64_t k_stride[4],
+                  const int64_t v_stride[4], const int64_t do_stride[4],
+                  const int64_t dq_stride[4], const int64_t dk_stride[4],
+                  const int64_t dv_stride[4], int mask_kind, int dtype,
+                  const void* q, const void* k, const void* v, const void* dout,
+                  const void* dq, const void* dk, const void* dv);
 
 /* Size of the fixed device scratch array of sdpa_decode_fwd_noalloc(). */
 #define SDPA_NOALLOC_SCRATCH_BYTES (32u << 20)

@@ -62,6 +62,10 @@ _SIGNATURES = {
         + [ctypes.c_void_p, _I64x4]
         + [ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
     ),
+    "sdpa_bwd_plan": (
+        ctypes.c_int,
+        [ctypes.c_int] * 7 + [_I64x4] * 7 + [ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 7,
+    ),
     "sdpa_last_launch_count": (ctypes.c_int, []),
     "sdpa_take_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int)]),
     "sdpa_decode_fwd_noalloc": (
@@ -335,6 +339,22 @@ def sdpa_backward(
         )
     _check(status, "sdpa_bwd")
     return dq, dk, dv
+
+
+def backward_plan(query, key, value, grad, *, layout="bhle", mask_kind=MASK_NONE) -> str:
+    """Name of the kernel family sdpa_backward() would run for these tensors
+    (gradients laid out like their inputs)."""
+    lib = load_library()
+    B, Hq, L, E = _dims(query, layout)
+    _, Hkv, S, _ = _dims(key, layout)
+    Ev = _dims(value, layout)[3]
+    st = [_i64x4(_strides(t, layout)) for t in (query, key, value, grad, query, key, value)]
+    r = lib.sdpa_bwd_plan(B, Hq, Hkv, L, S, E, Ev, *st, mask_kind, _DTYPE_CODE[query.dtype],
+                          query.data_ptr(), key.data_ptr(), value.data_ptr(), grad.data_ptr(),
+                          query.data_ptr(), key.data_ptr(), value.data_ptr())
+    if r < 0:
+        _check(-r, "sdpa_bwd_plan")
+    return {1: "backward_tcgen05", 3: "backward_simt"}[r]
 
 
 class _Attention(torch.autograd.Function):

@@ -260,12 +260,28 @@ static cudaError_t launch_backward_t(const Params& p, const BwdParams& g, cudaSt
   return cudaGetLastError();
 }
 
+template <typename T>
+static cudaError_t launch_rowdot_t(const Params& p, const BwdParams& g, cudaStream_t st) {
+  bwd_rowdot_kernel<T><<<dim3((p.L + kBwdWarps - 1) / kBwdWarps, p.Hq, p.B), kBwdWarps * 32, 0, st>>>(p, g);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_backward(const Params& p, const BwdParams& g, int dtype, cudaStream_t st, int* launches) {
   *launches = (p.L > 0 ? 2 : 0) + (p.S > 0 ? 1 : 0);
   switch (dtype) {
     case SDPA_F32: return launch_backward_t<float>(p, g, st);
     case SDPA_F16: return launch_backward_t<__half>(p, g, st);
     default: return launch_backward_t<__nv_bfloat16>(p, g, st);
+  }
+}
+
+// Only the row dot products D (for the tensor-core backward kernels).
+cudaError_t launch_rowdot(const Params& p, const BwdParams& g, int dtype, cudaStream_t st) {
+  if (p.L == 0) return cudaSuccess;
+  switch (dtype) {
+    case SDPA_F32: return launch_rowdot_t<float>(p, g, st);
+    case SDPA_F16: return launch_rowdot_t<__half>(p, g, st);
+    default: return launch_rowdot_t<__nv_bfloat16>(p, g, st);
   }
 }
 

@@ -16,6 +16,10 @@ cudaError_t launch_prefill(const Params& p, int dtype, cudaStream_t st);
 cudaError_t prefill_take_error(int* code);
 cudaError_t launch_backward(const Params& p, const BwdParams& g, int dtype, cudaStream_t st, int* launches);
 size_t backward_workspace_bytes(int B, int Hq, int L);
+cudaError_t launch_rowdot(const Params& p, const BwdParams& g, int dtype, cudaStream_t st);
+bool backward_sm100_supported(const Params& p, const BwdParams& g, int dtype);
+cudaError_t launch_backward_sm100(const Params& p, const BwdParams& g, int dtype, cudaStream_t st);
+cudaError_t backward_take_error(int* code);
 }  // namespace sdpa15
 
 using namespace sdpa15;
@@ -102,7 +106,10 @@ int sdpa_take_device_error(int* code) {
   if (!code) return SDPA_ERR_INVALID;
   *code = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return SDPA_ERR_CUDA;
-  return prefill_take_error(code) == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+  int c1 = 0, c2 = 0;
+  if (prefill_take_error(&c1) != cudaSuccess || backward_take_error(&c2) != cudaSuccess) return SDPA_ERR_CUDA;
+  *code = c1 ? c1 : c2;
+  return SDPA_OK;
 }
 
 size_t sdpa_fwd_workspace_size(int B, int Hq, int Hkv, int L, int S, int E, int Ev, int mask_kind,
@@ -250,10 +257,43 @@ int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const
   }
   g.D = static_cast<float*>(workspace);
   int launches = 0;
-  if (launch_backward(p, g, dtype, static_cast<cudaStream_t>(stream), &launches) != cudaSuccess)
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (backward_sm100_supported(p, g, dtype)) {
+    if (launch_rowdot(p, g, dtype, cs) != cudaSuccess || launch_backward_sm100(p, g, dtype, cs) != cudaSuccess)
+      return SDPA_ERR_CUDA;
+    launches = 3;
+  } else if (launch_backward(p, g, dtype, cs, &launches) != cudaSuccess) {
     return SDPA_ERR_CUDA;
+  }
   t_last_launches = launches;
   return SDPA_OK;
+}
+
+int sdpa_bwd_plan(int B, int Hq, int Hkv, int L, int S, int E, int Ev, const int64_t q_stride[4],
+                  const int64_t k_stride[4], const int64_t v_stride[4], const int64_t do_stride[4],
+                  const int64_t dq_stride[4], const int64_t dk_stride[4], const int64_t dv_stride[4],
+                  int mask_kind, int dtype, const void* q, const void* k, const void* v, const void* dout,
+                  const void* dq, const void* dk, const void* dv) {
+  int st = check_shapes(B, Hq, Hkv, L, S, E, Ev, q_stride, k_stride, v_stride, do_stride, mask_kind, dtype);
+  if (st == SDPA_OK)
+    st = check_shapes(B, Hq, Hkv, L, S, E, Ev, dq_stride, dk_stride, dv_stride, do_stride, mask_kind, dtype);
+  if (st != SDPA_OK) return -st;
+  Params p;
+  fill_params(p, q, k, v, nullptr, nullptr, B, Hq, Hkv, L, S, E, Ev, q_stride, k_stride, v_stride, do_stride,
+              mask_kind);
+  BwdParams g;
+  memset(&g, 0, sizeof(g));
+  g.dO = dout;
+  g.dq = const_cast<void*>(dq);
+  g.dk = const_cast<void*>(dk);
+  g.dv = const_cast<void*>(dv);
+  for (int d = 0; d < 4; ++d) {
+    g.dos[d] = do_stride[d];
+    g.dqs[d] = dq_stride[d];
+    g.dks[d] = dk_stride[d];
+    g.dvs[d] = dv_stride[d];
+  }
+  return backward_sm100_supported(p, g, dtype) ? kPlanPrefill : kPlanSimt;
 }
 
 }  // extern "C"

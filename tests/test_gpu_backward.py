@@ -72,6 +72,9 @@ CASES = [
     (torch.float16, 1, 2, 2, 40, 200, 64, 32, False),
     (torch.bfloat16, 1, 2, 1, 300, 100, 128, 128, True),   # L > S: rows past S keep every key
     (torch.float16, 1, 1, 1, 1, 64, 256, 256, False),      # one query row, widest head
+    (torch.float16, 1, 2, 2, 17, 400, 96, 96, False),      # few rows, several key tiles, ragged
+    (torch.bfloat16, 2, 4, 2, 700, 700, 128, 128, True),   # several tiles both ways, GQA
+    (torch.bfloat16, 1, 2, 2, 129, 640, 64, 64, True),     # causal with S > L
 ]
 
 
@@ -80,6 +83,11 @@ def test_backward_small(case):
     dt, B, Hq, Hkv, L, S, E, Ev, causal = case
     q, k, v = W.randn((B, Hq, L, E), 401, dt), W.randn((B, Hkv, S, E), 402, dt), W.randn((B, Hkv, S, Ev), 403, dt)
     g = W.randn((B, Hq, L, Ev), 404, dt)
+    from scaled_dot_product_15_b200.api import backward_plan
+
+    want = "backward_tcgen05" if (dt != torch.float32 and E == Ev and E in (64, 96, 128)) else "backward_simt"
+    qd = q.to(DEV)
+    assert backward_plan(qd, k.to(DEV), v.to(DEV), g.to(DEV), mask_kind=1 if causal else 0) == want
     got = _run(q, k, v, g, is_causal=causal, enable_gqa=Hq != Hkv)
     ref = ref_bwd(q, k, v, g, is_causal=causal, enable_gqa=Hq != Hkv)
     _check(got, ref, dt, str(case))
