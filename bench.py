@@ -509,6 +509,8 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=2.0, help="oracle seconds per reference step")
     ap.add_argument("--bare", action="store_true",
                     help="only run the workload's launches (for profilers); prints no bench line")
+    ap.add_argument("--bare-backward", action="store_true",
+                    help="time only the workload's backward (gradients) and print one short line (for profilers)")
     ap.add_argument("--bare-batch", type=int, default=0,
                     help="with --bare: use this batch size instead of the workload's (smaller profiler captures)")
     args = ap.parse_args()
@@ -528,6 +530,11 @@ def main():
     load_library()
     peaks, peak_src = load_peaks()
     w = W.WORKLOADS[args.workload]
+    if args.bare_backward:
+        r = measure_backward(w, args.steps, args.warmup, peaks, peak_src, device)
+        print(json.dumps({"bare_backward": w.name, "ms_per_step": r["ms_per_step"], "path": r["path"],
+                          "launches": r["gpu_launches"]}))
+        return
     if args.bare:
         if args.bare_batch:
             import dataclasses
