@@ -76,6 +76,31 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_rowdot_kernel(Params p, Bw
   if (lane == 0) g.D[((int64_t)b * p.Hq + h) * p.L + i] = acc;
 }
 
+// The same with 16-byte loads: LPR lanes (a power of two, LPR * 8 >= Ev)
+// share a row, 32 / LPR rows per warp.  For 16-bit types with Ev % 8 == 0
+// and 16-byte aligned rows.
+template <typename T, int LPR>
+__global__ void __launch_bounds__(kBwdWarps * 32) bwd_rowdot_vec_kernel(Params p, BwdParams g) {
+  constexpr int kRows = 32 / LPR;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = (blockIdx.x * kBwdWarps + warp) * kRows + lane / LPR, h = blockIdx.y, b = blockIdx.z;
+  const int c = lane % LPR;  // 8-element chunk of the row
+  float acc = 0.f;
+  if (i < p.L && c * 8 < p.Ev) {
+    const T* op = static_cast<const T*>(p.o) + b * p.os[0] + h * p.os[1] + (int64_t)i * p.os[2];
+    const T* gp = static_cast<const T*>(g.dO) + b * g.dos[0] + h * g.dos[1] + (int64_t)i * g.dos[2];
+    const uint4 ov = *reinterpret_cast<const uint4*>(op + 8 * c);
+    const uint4 gv = *reinterpret_cast<const uint4*>(gp + 8 * c);
+    const T* oe = reinterpret_cast<const T*>(&ov);
+    const T* ge = reinterpret_cast<const T*>(&gv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc = fmaf(to_f32<T>(ge[e]), to_f32<T>(oe[e]), acc);
+  }
+#pragma unroll
+  for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (c == 0 && i < p.L) g.D[((int64_t)b * p.Hq + h) * p.L + i] = acc;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkdv_kernel(Params p, BwdParams g) {
   extern __shared__ float smem[];
@@ -260,9 +285,22 @@ static cudaError_t launch_backward_t(const Params& p, const BwdParams& g, cudaSt
   return cudaGetLastError();
 }
 
+template <typename T, int LPR>
+static void launch_rowdot_vec(const Params& p, const BwdParams& g, cudaStream_t st) {
+  constexpr int rows_per_block = kBwdWarps * (32 / LPR);
+  bwd_rowdot_vec_kernel<T, LPR>
+      <<<dim3((p.L + rows_per_block - 1) / rows_per_block, p.Hq, p.B), kBwdWarps * 32, 0, st>>>(p, g);
+}
+
 template <typename T>
 static cudaError_t launch_rowdot_t(const Params& p, const BwdParams& g, cudaStream_t st) {
-  bwd_rowdot_kernel<T><<<dim3((p.L + kBwdWarps - 1) / kBwdWarps, p.Hq, p.B), kBwdWarps * 32, 0, st>>>(p, g);
+  const bool vec = sizeof(T) == 2 && p.Ev % 8 == 0 && p.os[2] % 8 == 0 && g.dos[2] % 8 == 0 && p.os[1] % 8 == 0 &&
+                   g.dos[1] % 8 == 0 && p.os[0] % 8 == 0 && g.dos[0] % 8 == 0 &&
+                   (reinterpret_cast<uintptr_t>(p.o) & 15) == 0 && (reinterpret_cast<uintptr_t>(g.dO) & 15) == 0;
+  if (vec && p.Ev <= 64) launch_rowdot_vec<T, 8>(p, g, st);
+  else if (vec && p.Ev <= 128) launch_rowdot_vec<T, 16>(p, g, st);
+  else if (vec) launch_rowdot_vec<T, 32>(p, g, st);
+  else bwd_rowdot_kernel<T><<<dim3((p.L + kBwdWarps - 1) / kBwdWarps, p.Hq, p.B), kBwdWarps * 32, 0, st>>>(p, g);
   return cudaGetLastError();
 }
 

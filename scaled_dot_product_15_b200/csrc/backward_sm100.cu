@@ -101,7 +101,7 @@ template <int D>
 struct CfgK {
   static constexpr int T = Tile<D>::BYTES;
   static constexpr int K_OFF = 0, V_OFF = T, R_OFF = 2 * T;  // ring: 2 x (Q_i, grad_i)
-  static constexpr int VEC_OFF = 6 * T;                      // lse, D: [2 buffers][2][128] floats
+  static constexpr int VEC_OFF = 6 * T;                      // lse, D: [2 buffers][2 warpgroups][2][64] floats
   static constexpr int BAR_OFF = VEC_OFF + 2048;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
 };
@@ -147,12 +147,15 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d, uint64_t da, uint64_t db,
 }
 
 // Acc += A B over K = 128 with A (16-bit, packed two per column) in tensor
-// memory at a and B an MN-major shared-memory operand.
-template <int KK = 0>
+// memory at a and B an MN-major shared-memory operand.  kSplit: A's K
+// columns 0-63 are packed at a + [0, 32) and 64-127 at a + [64, 96) (each
+// warpgroup's own half of the columns it read).
+template <bool kSplit = false, int KK = 0>
 __device__ __forceinline__ void mma_tmem_a(uint32_t acc, uint32_t a, uint64_t db, uint32_t idesc, uint32_t acc0) {
   if constexpr (KK < BN / 16) {
-    ptx::mma_ts_off<KK * 8, ((KK * 16 * 128) >> 4)>(acc, a, db, idesc, KK > 0 ? 1u : acc0);
-    mma_tmem_a<KK + 1>(acc, a, db, idesc, acc0);
+    constexpr uint32_t col = kSplit ? (KK / 4) * 64 + (KK % 4) * 8 : KK * 8;
+    ptx::mma_ts_off<col, ((KK * 16 * 128) >> 4)>(acc, a, db, idesc, KK > 0 ? 1u : acc0);
+    mma_tmem_a<kSplit, KK + 1>(acc, a, db, idesc, acc0);
   }
 }
 
@@ -187,17 +190,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// Barrier over warps 0-7 (named barrier 1) that also ORs a flag over them,
-// so every thread takes the same decision after it.
-__device__ __forceinline__ bool barrier256_any(bool flag) {
+// Barrier over the four warps of warpgroup w (named barrier 1 + w) that
+// also ORs a flag over them, so every thread takes the same decision after it.
+__device__ __forceinline__ bool wg_barrier_any(int w, bool flag) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)flag)
+      : "r"((uint32_t)flag), "r"(1 + w)
       : "memory");
   return r != 0;
 }
@@ -545,8 +548,8 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           break;
         }
         ptx::tc_fence_after();
-        mma_tmem_a(tmem + 256, tmem, dgmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);        // dV += P^T grad_i
-        mma_tmem_a(tmem + 384, tmem + 128, dqmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);  // dK += dS^T Q_i
+        mma_tmem_a<true>(tmem + 256, tmem, dgmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);        // dV += P^T grad_i
+        mma_tmem_a<true>(tmem + 384, tmem + 128, dqmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);  // dK += dS^T Q_i
         ptx::mma_commit(&bars->qempty[slot]);
         if (it + 1 < iters) {
           // In issue order after the products that read P^T and dS^T.
@@ -569,7 +572,6 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ptx::regs_inc<kRegsWork>();
     // ------------------------------------------------------------ elementwise
     const int w = warp >> 2;                   // query columns 64w..64w+63
-    const int u = tid;                         // 0..255
     const int r = (warp & 3) * 32 + lane;      // key row within the tile
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const int kj = key0 + r;                   // key within the sequence
@@ -577,9 +579,11 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
       const int h = kvh * p.group + it / per, q0 = (qt_lo + it % per) * BM;
-      float* lv = vec + (it & 1) * 256;  // lse * log2(e) of the tile's query rows, then their D
-      if (u < 128) {
-        const int qi = q0 + u;
+      // lse * log2(e) and D of this warpgroup's 64 query rows, staged by its
+      // first 64 threads ([buffer][warpgroup][lse2 | D][64]).
+      float* lv = vec + ((it & 1) * 2 + w) * 128;
+      if (r < 64) {
+        const int qi = q0 + 64 * w + r;
         float l2 = INFINITY, dd = 0.f;  // rows past the end: weight 0
         if (qi < Lq) {
           const int64_t ridx = ((int64_t)sg.b * p.Hq + h) * p.L + sg.seq0 + qi;
@@ -587,8 +591,8 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;
           dd = g.D[ridx];
         }
-        lv[u] = l2;
-        lv[128 + u] = dd;
+        lv[r] = l2;
+        lv[64 + r] = dd;
       }
       ok = __all_sync(0xffffffffu, wait(bars, &bars->sdp_ready, it & 1));
       ptx::tc_fence_after();
@@ -600,11 +604,11 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ptx::tmem_ld32(tmem + lane_off + 128 + 64 * w + 32, dp[1]);
         ptx::tmem_wait_ld();
       }
-      // Every thread's S^T and dP^T columns are in registers, and lse / D
-      // are staged, before any packed result overwrites tensor memory.
-      // (every one of the 256 threads reaches this barrier on every
-      // iteration, and all leave together if any of them timed out)
-      if (barrier256_any(!ok)) {
+      // The staged lse / D are visible to the warpgroup (every one of its
+      // 128 threads reaches this barrier on every iteration, and all leave
+      // together if any of them timed out).  Each thread packs its results
+      // over columns it has read itself, so no other warpgroup is waited for.
+      if (wg_barrier_any(w, !ok)) {
         ok = false;
         break;
       }
@@ -618,19 +622,19 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int i = 16 * half + ii;
           const int c0 = 2 * i, c1 = 2 * i + 1;
           const int q_0 = 64 * w + c0, q_1 = 64 * w + c1;
-          float p0 = exp2f_fast(__uint_as_float(s[c0 >> 5][c0 & 31]) * sl - lv[q_0]);
-          float p1 = exp2f_fast(__uint_as_float(s[c1 >> 5][c1 & 31]) * sl - lv[q_1]);
+          float p0 = exp2f_fast(__uint_as_float(s[c0 >> 5][c0 & 31]) * sl - lv[c0]);
+          float p1 = exp2f_fast(__uint_as_float(s[c1 >> 5][c1 & 31]) * sl - lv[c1]);
           if (masked) {
             if (kj >= Sk || (causal && kj > q0 + q_0)) p0 = 0.f;
             if (kj >= Sk || (causal && kj > q0 + q_1)) p1 = 0.f;
           }
-          const float d0 = p0 * (__uint_as_float(dp[c0 >> 5][c0 & 31]) - lv[128 + q_0]);
-          const float d1 = p1 * (__uint_as_float(dp[c1 >> 5][c1 & 31]) - lv[128 + q_1]);
+          const float d0 = p0 * (__uint_as_float(dp[c0 >> 5][c0 & 31]) - lv[64 + c0]);
+          const float d1 = p1 * (__uint_as_float(dp[c1 >> 5][c1 & 31]) - lv[64 + c1]);
           pp[ii] = pack2<T>(p0, p1);
           dsp[ii] = pack2<T>(d0, d1);
         }
-        tmem_st16(tmem + lane_off + 32 * w + 16 * half, pp);
-        tmem_st16(tmem + lane_off + 128 + 32 * w + 16 * half, dsp);
+        tmem_st16(tmem + lane_off + 64 * w + 16 * half, pp);
+        tmem_st16(tmem + lane_off + 128 + 64 * w + 16 * half, dsp);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();

@@ -33,7 +33,7 @@
 //   warps 0-7   softmax, one thread per query row (warpgroup i owns sub-tile
 //               i): tcgen05.ld of its 128 scores, masking on boundary tiles
 //               only, row maximum, exp2 with scale*log2(e) folded into one
-//               packed FMA (2 of every 8 pairs on the FMA pipe), P packed to
+//               packed FMA (1 of every 8 pairs on the FMA pipe), P packed to
 //               16 bits and stored over its own scores.  The output is
 //               rescaled in tensor memory only when a row maximum grows by more
 //               than 2^8 (exact: the final normalisation uses the same
@@ -87,6 +87,12 @@ constexpr int kRegsLaunch = (65536 / kThreads) / 8 * 8;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * kRegsLaunch, "register split");
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
+// Exponential pairs of every 8 computed on the FMA pipe instead of the
+// multi-function unit.
+#ifndef PF_EMU
+#define PF_EMU 1
+#endif
+constexpr int kEmuPer8 = PF_EMU;
 
 template <int D>
 struct Cfg {
@@ -147,6 +153,20 @@ __device__ __forceinline__ bool wait(Bars* bars, uint64_t* bar, uint32_t parity)
   return ptx::mbar_wait(bar, parity, kTimeoutNs, &bars->abort);
 }
 
+// Wait of the producer, which runs ahead: polls with a short sleep in
+// between, leaving issue slots to the softmax warps of its sub-partition.
+__device__ __forceinline__ bool wait_idle(Bars* bars, uint64_t* bar, uint32_t parity) {
+  const uint32_t a = ptx::smem_u32(bar);
+  if (ptx::mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (;;) {
+    __nanosleep(128);
+    if (ptx::mbar_try_wait(a, parity)) return true;
+    if (*reinterpret_cast<const volatile int*>(&bars->abort) != 0) return false;
+    if (ptx::globaltimer_ns() - t0 > kTimeoutNs) return false;
+  }
+}
+
 // Wait for this thread's own asynchronous copies or MMAs to finish before the
 // CTA exits: bounded, but not cut short by another role's abort.
 __device__ __forceinline__ bool drain(uint64_t* bar, uint32_t parity) {
@@ -203,7 +223,7 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[4][32]) {
 // P = 2^(S * scale*log2(e) - m) for 128 scores, two at a time (packed fp32
 // FMA), packed to 16-bit pairs in place over the scores (lower key in the low
 // half) and stored over S in tensor memory; returns the row sum of the fp32
-// weights.  With kEmu, 2 of every 8 pairs take the FMA-pipe 2^x so the
+// weights.  With kEmu, kEmuPer8 of every 8 pairs take the FMA-pipe 2^x so the
 // multi-function unit is not the bottleneck; masked tiles (-inf scores) use
 // the multi-function unit only, whose 2^-inf is exactly 0.
 template <typename T, bool kEmu>
@@ -220,7 +240,7 @@ __device__ __forceinline__ float exp_pack_store(uint32_t (&s)[4][32], float sl, 
                                sl2, nm2);
       float x0, x1, p0, p1;
       upk(x, x0, x1);
-      if (kEmu && (i % 8) < 2) {
+      if (kEmu && (i % 8) < kEmuPer8) {
         exp2_pair(x0, x1, p0, p1);
       } else {
         p0 = ptx::ex2(x0);
@@ -416,7 +436,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               if (!ok) break;
             }
             const int slot = t % C::NS;
-            if (!wait(bars, &bars->empty[slot], ((t / C::NS) & 1) ^ 1)) {
+            if (!wait_idle(bars, &bars->empty[slot], ((t / C::NS) & 1) ^ 1)) {
               ok = false;
               break;
             }
