@@ -452,6 +452,21 @@ def cpu_baseline(w: W.Workload, seconds: float):
 # ----------------------------------------------------------------- main
 
 
+def max_over_ranks(x: float, device, dist_on: bool) -> float:
+    """The largest of every rank's `x` (every rank gets it): the job is as
+    slow as its slowest rank."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if dist_on:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(amount_per_rank: float, ranks: int, max_ms_per_step: float, unit: str) -> float:
+    """Whole-job throughput: the work of every rank over the slowest rank's
+    time per step (weak scaling: each rank runs its own replica)."""
+    return rate(amount_per_rank * ranks, max_ms_per_step, unit)
+
+
 def dist_setup(n_gpus):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -548,17 +563,11 @@ def main():
     sampler = ClockSampler(local)
     res, total_ms, kernel_ms, launches = measure_workload(w, args.steps, args.warmup, peaks, peak_src, device,
                                                          dist_on, sampler)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if dist_on:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(total_ms, device, dist_on)
     amount, unit, _ = work_units(w)
-    value = rate(amount * ws, max_ms / args.steps, unit)
+    value = job_rate(amount, ws, max_ms / args.steps, unit)
     e2e_ms, h2d, d2h = time_e2e(w, [W.make_inputs(w, device)], max(3, args.steps // 10), 3)
-    t2 = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if dist_on:
-        torch.distributed.all_reduce(t2, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = rate(amount * ws, float(t2.item()), unit)
+    e2e_value = job_rate(amount, ws, max_over_ranks(e2e_ms, device, dist_on), unit)
 
     extra = {}
     cpu = None
