@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
   SDPA_OK = 0,
   SDPA_ERR_INVALID = 1,     /* bad argument: null pointer, shape, stride, GQA ratio, cu_seqlens, dtype */
-  SDPA_ERR_UNSUPPORTED = 2, /* well-formed but not implemented: E or Ev outside 1..256, not an sm_100 device */
+  SDPA_ERR_UNSUPPORTED = 2, /* well-formed but not implemented: E outside 0..256 or Ev outside 1..256, not an sm_100 device */
   SDPA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   SDPA_ERR_WORKSPACE = 4    /* workspace missing or smaller than sdpa_fwd_workspace_size() */
 } sdpa_status;
@@ -94,6 +94,9 @@ size_t sdpa_fwd_workspace_size(int B, int Hq, int Hkv, int L, int S, int E, int 
  * dtype             SDPA_F32, SDPA_F16 or SDPA_BF16 (q, k, v and out share it)
  * has_scale, scale  has_scale == 0: scale = 1/sqrt(E); else `scale` as given
  *                   (any finite value, 0 included)
+ * E = 0             allowed: the scores are empty sums, so the logits are
+ *                   the mask alone (exactref "Full specification"); q and k
+ *                   may then be NULL.
  * mask_kind         sdpa_mask_kind
  * cu_seqlens        BLOCK_DIAG*: device int32[n_seqs + 1], cumulative segment
  *                   starts of one packed batch: cu[0] = 0, non-decreasing,
@@ -187,7 +190,7 @@ size_t sdpa_bwd_workspace_size(int B, int Hq, int Hkv, int L, int S, int E, int 
  * the gradients.  Kernels: a row-dot kernel for D, then either the tcgen05
  * dK/dV and dQ kernels (see sdpa_bwd_plan) or the general SIMT ones; each
  * output element is written once, so results are deterministic.  Returns SDPA_OK, SDPA_ERR_INVALID (shapes, strides,
- * pointers), SDPA_ERR_UNSUPPORTED (head sizes outside 1..256, not an sm_100
+ * pointers), SDPA_ERR_UNSUPPORTED (E outside 0..256, Ev outside 1..256, not an sm_100
  * device), SDPA_ERR_WORKSPACE or SDPA_ERR_CUDA.
  */
 int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,

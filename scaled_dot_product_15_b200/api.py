@@ -165,7 +165,8 @@ def sdpa(
     """softmax(Q K^T * scale + mask) V and the per-row logsumexp, on a B200.
 
     ``layout="bhle"``: tensors are (B, H, L, E); ``"bmhk"``: (B, L, H, E), the
-    xFormers layout.  With ``cu_seqlens`` (int32, on the device, n+1 cumulative
+    xFormers layout; ``"bmghk"``: the xFormers grouped layout (B, L, G, H, E)
+    with key/value broadcast over H (see _sdpa_bmghk).  With ``cu_seqlens`` (int32, on the device, n+1 cumulative
     segment starts) the inputs are one packed batch (1, T, H, E) attended
     block-diagonally, causally within each segment when ``is_causal``.
     Returns ``(out, lse)``: out in the query's layout with Ev features, lse
@@ -173,6 +174,8 @@ def sdpa(
     """
     if dropout_p != 0.0:
         raise ValueError("dropout is random and has no reference; dropout_p must be 0")
+    if layout == "bmghk":
+        return _sdpa_bmghk(query, key, value, attn_mask, is_causal, scale, out, lse)
     lib = load_library()
     if query.dim() != 4 or key.dim() != 4 or value.dim() != 4:
         raise ValueError("query, key and value must be 4-D")
@@ -382,6 +385,32 @@ def attention(query, key, value, is_causal=False, scale=None, enable_gqa=False, 
     """sdpa() as a differentiable op: returns the output; its backward runs
     sdpa_backward() (the logsumexp is kept for it, not differentiated)."""
     return _Attention.apply(query, key, value, is_causal, scale, enable_gqa, layout, cu_seqlens, max_seqlen)[0]
+
+
+def _sdpa_bmghk(query, key, value, attn_mask, is_causal, scale, out, lse):
+    """The xFormers BMGHK layout (insureai360 tutorial, section 5
+    "Grouped-query attention"): query (B, M, G, H, K); key and value
+    (B, M, G, H, K) with the H axis a broadcast (stride 0) or of extent 1, so
+    that query head (g, h) reads key/value group g.  Views only: the query's
+    (G, H) axes merge into G*H heads and the key/value's H axis is dropped,
+    which is exactly the contiguous GQA grouping the kernels implement.
+    Returns out (B, M, G, H, Kv) and lse (B, G, H, M)."""
+    for t in (query, key, value):
+        if t.dim() != 5:
+            raise ValueError("bmghk tensors must be 5-D")
+    B, M, G, H, K = query.shape
+    if query.stride(2) != H * query.stride(3):
+        raise ValueError("the query's G and H axes must be mergeable (stride_G == H * stride_H)")
+    if key.shape[2] != G or value.shape[2] != G:
+        raise ValueError("key/value must have the query's G axis")
+    q4 = query.reshape(B, M, G * H, K) if query.is_contiguous() else query.view(B, M, G * H, K)
+    k4 = key[:, :, :, 0, :]
+    v4 = value[:, :, :, 0, :]
+    o4 = None if out is None else out.view(B, M, G * H, value.shape[-1])
+    l3 = None if lse is None else lse.view(B, G * H, M)
+    o, l = sdpa(q4, k4, v4, attn_mask=attn_mask, is_causal=is_causal, scale=scale, enable_gqa=H > 1,
+                layout="bmhk", out=o4, lse=l3)
+    return o.view(B, M, G, H, value.shape[-1]), l.view(B, G, H, M)
 
 
 def plan(query, key, value, *, layout="bhle", mask_kind=MASK_NONE, out=None) -> str:

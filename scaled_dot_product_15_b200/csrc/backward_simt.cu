@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkdv_kernel(Params p, BwdP
         }
         dot = warp_sum(dot);
         dpd = warp_sum(dpd);
-        float logit = dot * p.scale;
+        float logit = p.E == 0 ? 0.f : dot * p.scale;  // E = 0: empty sums
         if (biasb) logit += __ldg(biasb + (int64_t)i * p.bs[2] + (int64_t)j * p.bs[3]);
         const float pij = weight(logit, s_lse[ii]);
         const float ds = pij * (dpd - s_D[ii]);
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dq_kernel(Params p, BwdPar
       }
       dot = warp_sum(dot);
       dpd = warp_sum(dpd);
-      float logit = dot * p.scale;
+      float logit = p.E == 0 ? 0.f : dot * p.scale;  // E = 0: empty sums
       if (biasp) logit += __ldg(biasp + (int64_t)j * p.bs[3]);
       const float ds = weight(logit, lse) * (dpd - Di);
 #pragma unroll

@@ -42,7 +42,7 @@ int check_shapes(int B, int Hq, int Hkv, int L, int S, int E, int Ev, const int6
   if (B < 0 || Hq < 0 || Hkv < 0 || L < 0 || S < 0 || E < 0 || Ev < 0) return SDPA_ERR_INVALID;
   if (Hkv == 0 || Hq == 0 || Hq % Hkv != 0) return SDPA_ERR_INVALID;
   if (B > 65535 || Hq > 65535) return SDPA_ERR_UNSUPPORTED;
-  if (E == 0 || E > 256 || Ev == 0 || Ev > 256) return SDPA_ERR_UNSUPPORTED;
+  if (E > 256 || Ev == 0 || Ev > 256) return SDPA_ERR_UNSUPPORTED;
   if (!qs || !ks || !vs || !os) return SDPA_ERR_INVALID;
   if (qs[3] != 1 || ks[3] != 1 || vs[3] != 1 || os[3] != 1) return SDPA_ERR_INVALID;
   for (int d = 0; d < 3; ++d)
@@ -62,7 +62,7 @@ void fill_params(Params& p, const void* q, const void* k, const void* v, void* o
   p.group = Hq / Hkv;
   for (int d = 0; d < 4; ++d) { p.qs[d] = qs[d]; p.ks[d] = ks[d]; p.vs[d] = vs[d]; p.os[d] = os[d]; }
   p.mask = mask;
-  p.scale = (float)(1.0 / sqrt((double)E));  // the default; sdpa_fwd() sets the real one
+  p.scale = E > 0 ? (float)(1.0 / sqrt((double)E)) : 1.f;  // the default; sdpa_fwd() sets the real one
   p.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
 }
 
@@ -147,7 +147,8 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   if (st != SDPA_OK) return st;
   if (has_scale && !isfinite(scale)) return SDPA_ERR_INVALID;
   if (B == 0 || L == 0) return SDPA_OK;  // nothing to compute
-  if (!q || !k || !v || !out || !lse) return SDPA_ERR_INVALID;
+  // With E = 0 the scores are empty sums: q and k hold no data.
+  if ((E > 0 && (!q || !k)) || !v || !out || !lse) return SDPA_ERR_INVALID;
   if (mask_kind == SDPA_MASK_BLOCK_DIAG || mask_kind == SDPA_MASK_BLOCK_DIAG_CAUSAL) {
     if (!cu_seqlens || n_seqs < 1 || max_seqlen < 1) return SDPA_ERR_INVALID;
   }
@@ -161,7 +162,7 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   Params p;
   fill_params(p, q, k, v, out, lse, B, Hq, Hkv, L, S, E, Ev, q_stride, k_stride, v_stride, o_stride,
               mask_kind);
-  p.scale = has_scale ? scale : (float)(1.0 / sqrt((double)E));
+  p.scale = has_scale ? scale : (E > 0 ? (float)(1.0 / sqrt((double)E)) : 1.f);
   p.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   p.cu = cu_seqlens;
   p.n_seqs = n_seqs;
@@ -216,7 +217,8 @@ int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const
   if (st != SDPA_OK) return st;
   if (has_scale && !isfinite(scale)) return SDPA_ERR_INVALID;
   if (B == 0) return SDPA_OK;
-  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return SDPA_ERR_INVALID;
+  // With E = 0, q, k, dq and dk hold no data.
+  if ((E > 0 && (!q || !k || !dq || !dk)) || !v || !out || !lse || !dout || !dv) return SDPA_ERR_INVALID;
   if (mask_kind == SDPA_MASK_BLOCK_DIAG || mask_kind == SDPA_MASK_BLOCK_DIAG_CAUSAL) {
     if (!cu_seqlens || n_seqs < 1 || max_seqlen < 1) return SDPA_ERR_INVALID;
   }
@@ -234,7 +236,7 @@ int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const
   Params p;
   fill_params(p, q, k, v, const_cast<void*>(out), const_cast<float*>(lse), B, Hq, Hkv, L, S, E, Ev, q_stride,
               k_stride, v_stride, o_stride, mask_kind);
-  p.scale = has_scale ? scale : (float)(1.0 / sqrt((double)E));
+  p.scale = has_scale ? scale : (E > 0 ? (float)(1.0 / sqrt((double)E)) : 1.f);
   p.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   p.cu = cu_seqlens;
   p.n_seqs = n_seqs;

@@ -63,7 +63,7 @@ def test_host_side_rejections():
     assert _call(Hq=3, Hkv=2) == api.SDPA_ERR_INVALID          # Hq not a multiple of Hkv
     assert _call(dtype=7) == api.SDPA_ERR_INVALID               # unknown dtype
     assert _call(mask=9) == api.SDPA_ERR_INVALID                # unknown mask
-    assert _call(E=0) == api.SDPA_ERR_UNSUPPORTED               # E = 0 is not run on the GPU
+    assert _call(E=0, Ev=0) == api.SDPA_ERR_UNSUPPORTED         # Ev = 0: no output features
     assert _call(E=512) == api.SDPA_ERR_UNSUPPORTED
     assert _call(qstride=(1, 1, 1, 2)) == api.SDPA_ERR_INVALID  # feature stride must be 1
     assert _call(mask=api.MASK_BLOCK_DIAG, B=2) == api.SDPA_ERR_INVALID

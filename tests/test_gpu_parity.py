@@ -146,6 +146,52 @@ def test_prefill_row_maximum_moves_across_tiles(dt, causal, order):
     assert_close(out, lse, ro, rl, dt, f"{order} causal={causal}")
 
 
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_zero_head_size_logits_are_the_mask(dt):
+    """E = 0: the scores are empty sums, so the logits are the mask alone
+    (exactref "Full specification"); with no mask the weights are uniform."""
+    B, H, L, S, Ev = 1, 2, 40, 70, 32
+    q = torch.empty((B, H, L, 0), dtype=dt)
+    k = torch.empty((B, H, S, 0), dtype=dt)
+    v = _rand((B, H, S, Ev), 501, dt)
+    bias = W.randn((1, H, L, S), 502, torch.float32)
+    for kw in (dict(), dict(is_causal=True), dict(attn_mask=bias)):
+        out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), **kw)
+        ro, rl = ref_sdpa(q, k, v, **kw)
+        assert_close(out, lse, ro, rl, dt, f"E=0 {list(kw)}")
+    from oracle import sdpa_backward as ref_bwd
+    from scaled_dot_product_15_b200 import sdpa, sdpa_backward
+
+    g = _rand((B, H, L, Ev), 503, dt)
+    out, lse = sdpa(q.to(DEV), k.to(DEV), v.to(DEV), attn_mask=bias)
+    dq, dk, dv = sdpa_backward(q.to(DEV), k.to(DEV), v.to(DEV), out, lse, g.to(DEV), attn_mask=bias)
+    rq, rk, rv = ref_bwd(q, k, v, g, attn_mask=bias)
+    assert dq.shape == q.shape and dk.shape == k.shape
+    tol = (1e-4 if dt == torch.float32 else 2e-2) * max(1.0, float(np.abs(rv).max()))
+    assert float(np.abs(dv.double().cpu().numpy() - rv).max()) <= tol
+
+
+def test_bmghk_layout_is_grouped_query_attention():
+    """xFormers BMGHK (G key/value groups, H query heads per group, the key's
+    H axis broadcast) equals GQA with contiguous grouping, on the oracle."""
+    from scaled_dot_product_15_b200 import sdpa
+
+    dt = torch.bfloat16
+    B, M, G, H, K = 2, 300, 2, 4, 128
+    q = _rand((B, M, G, H, K), 511, dt)
+    kk = _rand((B, M, G, 1, K), 512, dt).expand(B, M, G, H, K)
+    vv = _rand((B, M, G, 1, K), 513, dt).expand(B, M, G, H, K)
+    out, lse = sdpa(q.to(DEV), kk.to(DEV), vv.to(DEV), is_causal=True, layout="bmghk")
+    torch.cuda.synchronize()
+    assert out.shape == (B, M, G, H, K) and lse.shape == (B, G, H, M)
+    # the oracle on (B, G*H, M, K) with key/value heads = G
+    qo = q.reshape(B, M, G * H, K).permute(0, 2, 1, 3)
+    ko = kk[:, :, :, 0].permute(0, 2, 1, 3)
+    vo = vv[:, :, :, 0].permute(0, 2, 1, 3)
+    ro, rl = ref_sdpa(qo, ko, vo, is_causal=True, enable_gqa=True)
+    assert_close(out.reshape(B, M, G * H, K).permute(0, 2, 1, 3), lse.reshape(B, G * H, M), ro, rl, dt, "bmghk")
+
+
 DECODE_CASES = [
     # dtype, B, Hq, Hkv, L, S, E
     (torch.bfloat16, 2, 8, 2, 1, 3000, 128),
