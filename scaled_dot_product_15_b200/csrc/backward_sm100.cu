@@ -36,6 +36,7 @@
 #include <algorithm>
 
 #include "backward.cuh"
+#include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
 #include "tma_host.cuh"
 
@@ -83,8 +84,8 @@ struct BarsQ {
 struct BarsK {
   uint64_t kv;                       // K and V tiles landed
   uint64_t qfull[2], qempty[2];      // (Q_i, grad_i) ring
-  uint64_t sdp_ready;                // S^T and dP^T computed (one phase per query tile)
-  uint64_t pds_ready;                // P^T and dS^T written
+  uint64_t sdp_ready[2];             // S^T and dP^T of query columns 64h..64h+63 computed
+  uint64_t pds_ready[2];             // warpgroup h's P^T and dS^T written
   uint64_t done;
   uint32_t tmem;
   int abort;
@@ -150,12 +151,13 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d, uint64_t da, uint64_t db,
 // memory at a and B an MN-major shared-memory operand.  kSplit: A's K
 // columns 0-63 are packed at a + [0, 32) and 64-127 at a + [64, 96) (each
 // warpgroup's own half of the columns it read).
-template <bool kSplit = false, int KK = 0>
+// KK in [KSTART, KEND) of the K = 128 products; the first one takes acc0.
+template <bool kSplit = false, int KSTART = 0, int KEND = BN / 16, int KK = KSTART>
 __device__ __forceinline__ void mma_tmem_a(uint32_t acc, uint32_t a, uint64_t db, uint32_t idesc, uint32_t acc0) {
-  if constexpr (KK < BN / 16) {
+  if constexpr (KK < KEND) {
     constexpr uint32_t col = kSplit ? (KK / 4) * 64 + (KK % 4) * 8 : KK * 8;
-    ptx::mma_ts_off<col, ((KK * 16 * 128) >> 4)>(acc, a, db, idesc, KK > 0 ? 1u : acc0);
-    mma_tmem_a<kSplit, KK + 1>(acc, a, db, idesc, acc0);
+    ptx::mma_ts_off<col, ((KK * 16 * 128) >> 4)>(acc, a, db, idesc, KK > KSTART ? 1u : acc0);
+    mma_tmem_a<kSplit, KSTART, KEND, KK + 1>(acc, a, db, idesc, acc0);
   }
 }
 
@@ -477,8 +479,10 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ptx::mbar_init(&bars->qfull[s], 1);
       ptx::mbar_init(&bars->qempty[s], 1);
     }
-    ptx::mbar_init(&bars->sdp_ready, 1);
-    ptx::mbar_init(&bars->pds_ready, 256);
+    for (int hf = 0; hf < 2; ++hf) {
+      ptx::mbar_init(&bars->sdp_ready[hf], 1);
+      ptx::mbar_init(&bars->pds_ready[hf], 128);
+    }
     ptx::mbar_init(&bars->done, 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
@@ -524,7 +528,12 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     } else if (warp == kWarpMma && lane == 0) {
       // ------------------------------------------------------------ MMA
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-      constexpr uint32_t idesc_s = ptx::idesc_f16(kBf16, BM, BN, false);
+      // Query columns are handled in two halves (64 each), one per
+      // elementwise warpgroup, so that one half's products overlap the other
+      // half's elementwise work: S^T / dP^T of a half are N = 64 products
+      // (the half's 64 query rows of Q_i / grad_i as B), dV / dK of a half
+      // the K = 64 slice of the query dimension.
+      constexpr uint32_t idesc_s = ptx::idesc_f16(kBf16, BM, BN / 2, false);
       constexpr uint32_t idesc_acc = ptx::idesc_f16(kBf16, BM, D, true);
       const uint64_t dk_ = ptx::sdesc_sw128(ptx::smem_u32(smem + C::K_OFF), 16, 1024);
       const uint64_t dv_ = ptx::sdesc_sw128(ptx::smem_u32(smem + C::V_OFF), 16, 1024);
@@ -534,35 +543,50 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint64_t dqmn = ptx::sdesc_sw128(r0, Tile<D>::BLOCK, 1024);          // Q_i, MN-major
       const uint64_t dgmn = ptx::sdesc_sw128(r0 + C::T, Tile<D>::BLOCK, 1024);   // grad_i, MN-major
       constexpr uint64_t kSlot = (2 * C::T) >> 4;
+      constexpr uint64_t kHalfRows = (64 * 128) >> 4;  // 64 rows of a 128-byte-row block
+      // S^T and dP^T of query half hf of the tile in ring slot ns.
+      auto scores = [&](int ns, int hf) {
+        const uint64_t off = ns * kSlot + hf * kHalfRows;
+        mma_kmajor<D>(tmem + 64 * hf, dk_, dq_ + off, idesc_s);
+        mma_kmajor<D>(tmem + 128 + 64 * hf, dv_, dg_ + off, idesc_s);
+        ptx::mma_commit(&bars->sdp_ready[hf]);
+      };
       bool ok = iters == 0 || (wait(bars, &bars->kv, 0) && wait(bars, &bars->qfull[0], 0));
       if (ok && iters > 0) {
         ptx::tc_fence_after();
-        mma_kmajor<D>(tmem, dk_, dq_, idesc_s);
-        mma_kmajor<D>(tmem + 128, dv_, dg_, idesc_s);
-        ptx::mma_commit(&bars->sdp_ready);
+        scores(0, 0);
+        scores(0, 1);
       }
       for (int it = 0; it < iters && ok; ++it) {
-        const int slot = it & 1;
-        if (!wait(bars, &bars->pds_ready, it & 1)) {
+        const int slot = it & 1, ns = (it + 1) & 1;
+        const bool next = it + 1 < iters;
+        // Half 0: dV += P^T grad_i and dK += dS^T Q_i over query rows 0-63,
+        // then (the next tile's Q_i and grad_i loaded) its next S^T, dP^T.
+        if (!wait(bars, &bars->pds_ready[0], it & 1)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        mma_tmem_a<true>(tmem + 256, tmem, dgmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);        // dV += P^T grad_i
-        mma_tmem_a<true>(tmem + 384, tmem + 128, dqmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);  // dK += dS^T Q_i
-        ptx::mma_commit(&bars->qempty[slot]);
-        if (it + 1 < iters) {
-          // In issue order after the products that read P^T and dS^T.
-          const int ns = (it + 1) & 1;
+        mma_tmem_a<true, 0, 4>(tmem + 256, tmem, dgmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);
+        mma_tmem_a<true, 0, 4>(tmem + 384, tmem + 128, dqmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);
+        if (next) {
           if (!wait(bars, &bars->qfull[ns], ((it + 1) >> 1) & 1)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          mma_kmajor<D>(tmem, dk_, dq_ + ns * kSlot, idesc_s);
-          mma_kmajor<D>(tmem + 128, dv_, dg_ + ns * kSlot, idesc_s);
-          ptx::mma_commit(&bars->sdp_ready);
+          scores(ns, 0);  // overwrites only half 0's columns
         }
+        // Half 1.
+        if (!wait(bars, &bars->pds_ready[1], it & 1)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        mma_tmem_a<true, 4, 8>(tmem + 256, tmem, dgmn + slot * kSlot, idesc_acc, 1u);
+        mma_tmem_a<true, 4, 8>(tmem + 384, tmem + 128, dqmn + slot * kSlot, idesc_acc, 1u);
+        ptx::mma_commit(&bars->qempty[slot]);
+        if (next) scores(ns, 1);
       }
       if (!ok) flag_error(bars, 23);
       ptx::mma_commit(&bars->done);
@@ -594,7 +618,7 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         lv[r] = l2;
         lv[64 + r] = dd;
       }
-      ok = __all_sync(0xffffffffu, wait(bars, &bars->sdp_ready, it & 1));
+      ok = __all_sync(0xffffffffu, wait(bars, &bars->sdp_ready[w], it & 1));
       ptx::tc_fence_after();
       uint32_t s[2][32], dp[2][32];
       if (ok) {
@@ -618,27 +642,39 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int half = 0; half < 2; ++half) {
         uint32_t pp[16], dsp[16];
 #pragma unroll
-        for (int ii = 0; ii < 16; ++ii) {
-          const int i = 16 * half + ii;
-          const int c0 = 2 * i, c1 = 2 * i + 1;
-          const int q_0 = 64 * w + c0, q_1 = 64 * w + c1;
-          float p0 = exp2f_fast(__uint_as_float(s[c0 >> 5][c0 & 31]) * sl - lv[c0]);
-          float p1 = exp2f_fast(__uint_as_float(s[c1 >> 5][c1 & 31]) * sl - lv[c1]);
-          if (masked) {
-            if (kj >= Sk || (causal && kj > q0 + q_0)) p0 = 0.f;
-            if (kj >= Sk || (causal && kj > q0 + q_1)) p1 = 0.f;
+        for (int qd = 0; qd < 8; ++qd) {  // 4 query columns at a time
+          const int c = 32 * half + 4 * qd;
+          const float4 l4 = *reinterpret_cast<const float4*>(lv + c);
+          const float4 d4 = *reinterpret_cast<const float4*>(lv + 64 + c);
+          const float ls[4] = {l4.x, l4.y, l4.z, l4.w}, ds[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int pr = 0; pr < 2; ++pr) {
+            const int c0 = c + 2 * pr, c1 = c0 + 1;
+            const float x0 = __uint_as_float(s[c0 >> 5][c0 & 31]) * sl - ls[2 * pr];
+            const float x1 = __uint_as_float(s[c1 >> 5][c1 & 31]) * sl - ls[2 * pr + 1];
+            float p0, p1;
+            if (pr == 1 && (qd & 1)) {
+              exp2poly::exp2_pair(x0, x1, p0, p1);  // 1 of 4 pairs on the FMA pipe
+            } else {
+              p0 = exp2f_fast(x0);
+              p1 = exp2f_fast(x1);
+            }
+            if (masked) {
+              if (kj >= Sk || (causal && kj > q0 + 64 * w + c0)) p0 = 0.f;
+              if (kj >= Sk || (causal && kj > q0 + 64 * w + c1)) p1 = 0.f;
+            }
+            const float d0 = p0 * (__uint_as_float(dp[c0 >> 5][c0 & 31]) - ds[2 * pr]);
+            const float d1 = p1 * (__uint_as_float(dp[c1 >> 5][c1 & 31]) - ds[2 * pr + 1]);
+            pp[2 * qd + pr] = pack2<T>(p0, p1);
+            dsp[2 * qd + pr] = pack2<T>(d0, d1);
           }
-          const float d0 = p0 * (__uint_as_float(dp[c0 >> 5][c0 & 31]) - lv[64 + c0]);
-          const float d1 = p1 * (__uint_as_float(dp[c1 >> 5][c1 & 31]) - lv[64 + c1]);
-          pp[ii] = pack2<T>(p0, p1);
-          dsp[ii] = pack2<T>(d0, d1);
         }
         tmem_st16(tmem + lane_off + 64 * w + 16 * half, pp);
         tmem_st16(tmem + lane_off + 128 + 64 * w + 16 * half, dsp);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->pds_ready);
+      ptx::mbar_arrive(&bars->pds_ready[w]);
     }
     // dk = scale * dK, dv = dV: warpgroup w writes the 32-column chunks c
     // with c % 2 == w of both.

@@ -154,7 +154,9 @@ class DqModel(_Hw):
 
 
 class DkdvModel(_Hw):
-    """dK/dV kernel: K and V once, a 2-slot ring of (Q_i, grad_i) tiles."""
+    """dK/dV kernel: K and V once, a 2-slot ring of (Q_i, grad_i) tiles; the
+    query columns in two halves, one per elementwise warpgroup, each with its
+    own S^T / dP^T columns (half h: 64h..64h+63) and barriers."""
 
     def __init__(self, iters, rng):
         super().__init__(rng)
@@ -163,11 +165,13 @@ class DkdvModel(_Hw):
         self.kv = B("kv", 1)
         self.qfull = [B(f"qfull{i}", 1) for i in range(2)]
         self.qempty = [B(f"qempty{i}", 1) for i in range(2)]
-        self.sdp_ready, self.pds_ready, self.done = B("sdp_ready", 1), B("pds_ready", 1), B("done", 1)
+        self.sdp_ready = [B(f"sdp_ready{h}", 1) for h in range(2)]
+        self.pds_ready = [B(f"pds_ready{h}", 1) for h in range(2)]
+        self.done = B("done", 1)
         self.slot = [None, None]
         self.slot_uses = {}   # tile -> products that read its slot
-        self.buf = None       # ("S", it) or ("P", it) in the S^T / dP^T columns
-        self.acc = []
+        self.buf = [None, None]  # per half: ("S", it) or ("P", it) or ("used", it)
+        self.acc = [[], []]
 
     def producer(self):
         self.tma.append(lambda: self.kv.arrive())
@@ -175,7 +179,7 @@ class DkdvModel(_Hw):
             s = it & 1
             yield ("wait", self.qempty[s], ((it >> 1) & 1) ^ 1, (it >> 1) - 1)
             old = self.slot[s]
-            if old is not None and self.slot_uses.get(old, 0) < 2:
+            if old is not None and self.slot_uses.get(old, 0) < 4:
                 raise ProtocolError(f"slot {s} refilled before tile {old} was fully read")
             self.slot[s] = None
 
@@ -184,23 +188,23 @@ class DkdvModel(_Hw):
                 self.qfull[s].arrive()
             self.tma.append(land)
 
-    def _sdp(self, it):
+    def _sdp(self, it, h):
         def f():
             if self.slot[it & 1] != it:
-                raise ProtocolError(f"S^T({it}) reads slot holding {self.slot[it & 1]}")
-            if self.buf is not None and self.buf[0] != "used":
-                raise ProtocolError(f"S^T({it}) overwrites {self.buf}")
+                raise ProtocolError(f"S^T({it},{h}) reads slot holding {self.slot[it & 1]}")
+            if self.buf[h] is not None and self.buf[h][0] != "used":
+                raise ProtocolError(f"S^T({it},{h}) overwrites {self.buf[h]}")
             self.slot_uses[it] = self.slot_uses.get(it, 0) + 1
-            self.buf = ("S", it)
+            self.buf[h] = ("S", it)
         return f
 
-    def _acc(self, it):
+    def _acc(self, it, h):
         def f():
-            if self.buf != ("P", it) or self.slot[it & 1] != it:
-                raise ProtocolError(f"dV/dK({it}) read {self.buf} and slot {self.slot[it & 1]}")
+            if self.buf[h] != ("P", it) or self.slot[it & 1] != it:
+                raise ProtocolError(f"dV/dK({it},{h}) read {self.buf[h]} and slot {self.slot[it & 1]}")
             self.slot_uses[it] = self.slot_uses.get(it, 0) + 1
-            self.buf = ("used", it)
-            self.acc.append(it)
+            self.buf[h] = ("used", it)
+            self.acc[h].append(it)
         return f
 
     def mma(self):
@@ -209,29 +213,35 @@ class DkdvModel(_Hw):
             return
         yield ("wait", self.kv, 0, 0)
         yield ("wait", self.qfull[0], 0, 0)
-        self.pipe += [("op", self._sdp(0)), ("commit", self.sdp_ready)]
+        for h in range(2):
+            self.pipe += [("op", self._sdp(0, h)), ("commit", self.sdp_ready[h])]
         for it in range(self.iters):
-            yield ("wait", self.pds_ready, it & 1, it)
-            self.pipe += [("op", self._acc(it)), ("commit", self.qempty[it & 1])]
-            if it + 1 < self.iters:
-                ns = (it + 1) & 1
+            nxt = it + 1 < self.iters
+            ns = (it + 1) & 1
+            yield ("wait", self.pds_ready[0], it & 1, it)
+            self.pipe.append(("op", self._acc(it, 0)))
+            if nxt:
                 yield ("wait", self.qfull[ns], ((it + 1) >> 1) & 1, (it + 1) >> 1)
-                self.pipe += [("op", self._sdp(it + 1)), ("commit", self.sdp_ready)]
+                self.pipe += [("op", self._sdp(it + 1, 0)), ("commit", self.sdp_ready[0])]
+            yield ("wait", self.pds_ready[1], it & 1, it)
+            self.pipe += [("op", self._acc(it, 1)), ("commit", self.qempty[it & 1])]
+            if nxt:
+                self.pipe += [("op", self._sdp(it + 1, 1)), ("commit", self.sdp_ready[1])]
         self.pipe.append(("commit", self.done))
 
-    def elementwise(self):
+    def elementwise(self, h):
         for it in range(self.iters):
-            yield ("wait", self.sdp_ready, it & 1, it)
-            if self.buf != ("S", it):
-                raise ProtocolError(f"elementwise({it}) reads {self.buf}")
-            self.buf = ("P", it)
-            self.pds_ready.arrive()
+            yield ("wait", self.sdp_ready[h], it & 1, it)
+            if self.buf[h] != ("S", it):
+                raise ProtocolError(f"elementwise({it},{h}) reads {self.buf[h]}")
+            self.buf[h] = ("P", it)
+            self.pds_ready[h].arrive()
         yield ("wait", self.done, 0, 0)
-        if self.acc != list(range(self.iters)):
-            raise ProtocolError(f"accumulated {self.acc}")
+        if self.acc[h] != list(range(self.iters)):
+            raise ProtocolError(f"accumulated {self.acc[h]}")
 
     def go(self):
-        self.run([self.producer(), self.mma(), self.elementwise()])
+        self.run([self.producer(), self.mma(), self.elementwise(0), self.elementwise(1)])
 
 
 @pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 7, 16])
@@ -257,9 +267,10 @@ def test_models_catch_mistakes():
     class EarlyQempty(DkdvModel):
         def mma(self):
             for item in DkdvModel.mma(self):
-                # release the slot as soon as S^T/dP^T were issued
-                if item[1] is self.pds_ready:
+                # release the slot after the first half's products only
+                if item[1] is self.pds_ready[1]:
                     self.pipe.append(("commit", self.qempty[item[3] & 1]))
+                    self.pipe[:] = [op for op in self.pipe[:-1] if not (op[0] == "commit" and op[1] in self.qempty)] + self.pipe[-1:]
                 yield item
 
     def caught(cls, arg):
