@@ -384,8 +384,8 @@ def measure_backward(w: W.Workload, steps: int, warmup: int, peaks, peak_src, de
         "path": path,
         "gpu_launches": launches,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None, "peak_source": f"of {peak_src}",
-                     "algorithmic_per_launch": amount},
+                     "frac": round(achieved / peak, 4), "traffic": stored_traffic(w.name + ":backward", path),
+                     "peak_source": f"of {peak_src}", "algorithmic_per_launch": amount},
         "note": "gradients (dq, dk, dv) of this workload: row-dot, dK/dV and dQ kernels",
     }
 
