@@ -147,8 +147,9 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   if (st != SDPA_OK) return st;
   if (has_scale && !isfinite(scale)) return SDPA_ERR_INVALID;
   if (B == 0 || L == 0) return SDPA_OK;  // nothing to compute
-  // With E = 0 the scores are empty sums: q and k hold no data.
-  if ((E > 0 && (!q || !k)) || !v || !out || !lse) return SDPA_ERR_INVALID;
+  // Tensors without elements may have NULL data: q and k when E = 0 (the
+  // scores are empty sums), k and v when S = 0 (every row keeps no key).
+  if ((E > 0 && !q) || (E > 0 && S > 0 && !k) || (S > 0 && !v) || !out || !lse) return SDPA_ERR_INVALID;
   if (mask_kind == SDPA_MASK_BLOCK_DIAG || mask_kind == SDPA_MASK_BLOCK_DIAG_CAUSAL) {
     if (!cu_seqlens || n_seqs < 1 || max_seqlen < 1) return SDPA_ERR_INVALID;
   }
@@ -217,8 +218,12 @@ int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const
   if (st != SDPA_OK) return st;
   if (has_scale && !isfinite(scale)) return SDPA_ERR_INVALID;
   if (B == 0) return SDPA_OK;
-  // With E = 0, q, k, dq and dk hold no data.
-  if ((E > 0 && (!q || !k || !dq || !dk)) || !v || !out || !lse || !dout || !dv) return SDPA_ERR_INVALID;
+  // Tensors without elements may have NULL data (E = 0: q, k, dq, dk;
+  // S = 0: k, v, dk, dv; L = 0: q, out, lse, dout, dq).
+  const bool rows = L > 0, keys = S > 0, feat = E > 0;
+  if ((rows && feat && (!q || !dq)) || (keys && feat && (!k || !dk)) || (keys && (!v || !dv)) ||
+      (rows && (!out || !lse || !dout)))
+    return SDPA_ERR_INVALID;
   if (mask_kind == SDPA_MASK_BLOCK_DIAG || mask_kind == SDPA_MASK_BLOCK_DIAG_CAUSAL) {
     if (!cu_seqlens || n_seqs < 1 || max_seqlen < 1) return SDPA_ERR_INVALID;
   }

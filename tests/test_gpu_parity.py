@@ -192,6 +192,64 @@ def test_bmghk_layout_is_grouped_query_attention():
     assert_close(out.reshape(B, M, G * H, K).permute(0, 2, 1, 3), lse.reshape(B, G * H, M), ro, rl, dt, "bmghk")
 
 
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_empty_dimensions(dt):
+    """No keys: every row has no kept key (out 0, lse -inf); no query rows or
+    no batch: nothing is written and nothing fails; the gradients of a
+    problem without keys are zero for the queries."""
+    from scaled_dot_product_15_b200 import sdpa, sdpa_backward
+
+    q = _rand((2, 3, 17, 64), 521, dt).to(DEV)
+    k0 = torch.empty((2, 3, 0, 64), dtype=dt, device=DEV)
+    v0 = torch.empty((2, 3, 0, 64), dtype=dt, device=DEV)
+    out, lse = _sdpa(q, k0, v0)
+    assert (out == 0).all() and torch.isneginf(lse).all()
+    g = _rand((2, 3, 17, 64), 522, dt).to(DEV)
+    dq, dk, dv = sdpa_backward(q, k0, v0, out, lse, g)
+    torch.cuda.synchronize()
+    assert (dq == 0).all() and dk.numel() == 0 and dv.numel() == 0
+    k = _rand((2, 3, 9, 64), 523, dt).to(DEV)
+    v = _rand((2, 3, 9, 64), 524, dt).to(DEV)
+    out, lse = _sdpa(q[:, :, :0], k, v)
+    assert out.shape == (2, 3, 0, 64) and lse.shape == (2, 3, 0)
+    dq, dk, dv = sdpa_backward(q[:, :, :0], k, v, out, lse, out)
+    torch.cuda.synchronize()
+    assert (dk == 0).all() and (dv == 0).all()
+    out, lse = _sdpa(q[:0], k[:0], v[:0])
+    assert out.numel() == 0
+
+
+BUDGET_CASES = [
+    # dtype, B, Hq, Hkv, L, S, E, causal
+    (torch.bfloat16, 1, 2, 2, 300, 300, 128, True),
+    (torch.float16, 1, 2, 2, 257, 257, 96, True),
+    (torch.bfloat16, 1, 8, 2, 200, 200, 128, False),
+    (torch.float16, 1, 2, 2, 200, 333, 64, False),
+    (torch.bfloat16, 2, 8, 2, 1, 3000, 128, False),   # decode kernel
+    (torch.float32, 1, 2, 2, 100, 77, 40, True),      # general kernel
+]
+
+
+@pytest.mark.parametrize("case", BUDGET_CASES, ids=lambda c: "-".join(str(x) for x in c))
+def test_within_the_error_budget(case):
+    """Element by element inside the per-element error budget of the
+    exactref tolerance model for the algorithm the kernels implement
+    (oracle/budget.py), which for 16-bit inputs is far sharper than the flat
+    2e-2."""
+    from oracle.budget import forward_budget
+
+    dt, B, Hq, Hkv, L, S, E, causal = case
+    q, k, v = _rand((B, Hq, L, E), 531, dt), _rand((B, Hkv, S, E), 532, dt), _rand((B, Hkv, S, E), 533, dt)
+    out, lse = _sdpa(q.to(DEV), k.to(DEV), v.to(DEV), is_causal=causal, enable_gqa=Hq != Hkv)
+    ro, rl = ref_sdpa(q, k, v, is_causal=causal, enable_gqa=Hq != Hkv)
+    name = {torch.float32: "float32", torch.float16: "float16", torch.bfloat16: "bfloat16"}[dt]
+    to, tl = forward_budget(q, k, v, dtype_name=name, is_causal=causal, enable_gqa=Hq != Hkv)
+    eo = np.abs(out.double().cpu().numpy() - ro)
+    el = np.abs(lse.double().cpu().numpy() - rl)
+    assert (eo <= to).all(), f"out outside the budget: max ratio {float((eo / to).max()):.2f}"
+    assert (el <= tl).all(), f"lse outside the budget: max ratio {float((el / tl).max()):.2f}"
+
+
 DECODE_CASES = [
     # dtype, B, Hq, Hkv, L, S, E
     (torch.bfloat16, 2, 8, 2, 1, 3000, 128),
