@@ -1,4 +1,5 @@
-"""Per-element error budgets for the attention forward (test infrastructure).
+"""Per-element error budgets for the attention forward and backward (test
+infrastructure).
 
 TEST INFRASTRUCTURE ONLY, like the rest of ``oracle/``: only tests use it.
 
@@ -31,8 +32,15 @@ element, for the algorithm the GPU kernels implement, evaluated on the exact
   P rounding, since the row sum uses the fp32 weights), the logarithm and
   the fp32 rounding of the sum.
 
-A ``safety`` factor (default 2) covers the second-order terms.  The budget is
-pinned in tests/test_budget_pins.py: an independent low-precision emulation
+``backward_budget`` does the same for the gradients of the FlashAttention
+backward: each recomputed weight inherits the logit error and the forward
+logsumexp's budget; D_i = grad_i . out_i the forward output's budget; dS the
+errors of dP, D and its cast; dQ, dK, dV the errors of their fp32 sums and the
+final rounding.
+
+A ``safety`` factor (default 2) covers the second-order terms.  The forward
+budget is pinned in tests/test_budget_pins.py, the backward one in
+tests/test_backward_budget_pins.py: an independent low-precision emulation
 of the algorithm stays inside it on random inputs, and planted mistakes (a
 scale off by 0.5 %, a dropped key, lse off by ulps of the dtype) leave it.
 """
@@ -44,7 +52,7 @@ import numpy as np
 
 from .sdpa_ref import _as_f64, _mask_to_bias, default_scale
 
-__all__ = ["unit_roundoff", "forward_budget"]
+__all__ = ["unit_roundoff", "forward_budget", "backward_budget"]
 
 _U32 = 2.0 ** -24
 
@@ -124,3 +132,91 @@ def forward_budget(
                 tl = (w * eta_sum).sum(axis=1) + 4 * _U32 + 2 * _U32 * np.abs(lse)
                 tol_l[b, h] = safety * tl
     return tol_o, tol_l
+
+
+def backward_budget(
+    query,
+    key,
+    value,
+    grad,
+    *,
+    dtype_name: str,
+    is_causal: bool = False,
+    scale: Optional[float] = None,
+    enable_gqa: bool = False,
+    exp_rel: Optional[float] = None,
+    safety: float = 2.0,
+) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """(tol_dq, tol_dk, tol_dv): per-element first-order bounds for the
+    gradients as the backward kernels compute them (the exactref backward
+    section's list: the forward's scores, scale, logits, shift, exp and row
+    sum; P; the accumulations of dP, D, grad_value, dS K and dS^T Q; the
+    roundings of dS and of the results), with the FlashAttention choices the
+    page names among the algorithms: P recomputed from the forward's fp32
+    logsumexp, P and dS cast to the input dtype before their products, and
+    D_i = grad_i . out_i taken from the forward's output in the input dtype."""
+    q, k, v, g = (_as_f64(x) for x in (query, key, value, grad))
+    B, Hq, L, E = q.shape
+    _, Hkv, S, _ = k.shape
+    Ev = v.shape[-1]
+    group = Hq // Hkv
+    s = default_scale(E) if scale is None else float(scale)
+    ud = unit_roundoff(dtype_name)
+    if exp_rel is None:
+        exp_rel = 1e-4 if dtype_name != "float32" else 4 * _U32
+    cast = ud if dtype_name != "float32" else 0.0
+    gE, gEv, gS, gL = (_gamma(max(n, 1), _U32) for n in (E, Ev, S, L * group))
+    # the forward's own errors enter through its output (D) and its
+    # logsumexp (every recomputed weight)
+    tol_o, tol_l = forward_budget(q, k, v, dtype_name=dtype_name, is_causal=is_causal, scale=scale,
+                                  enable_gqa=enable_gqa, exp_rel=exp_rel, safety=1.0)
+    tdq = np.zeros_like(q)
+    tdk = np.zeros_like(k)
+    tdv = np.zeros_like(v)
+    adk = np.zeros_like(k)  # sum of |terms| of dk, dv (for their accumulation errors)
+    adv = np.zeros_like(v)
+    dk_ex = np.zeros_like(k)
+    dv_ex = np.zeros_like(v)
+    with np.errstate(invalid="ignore", over="ignore", divide="ignore"):
+        for b in range(B):
+            for h in range(Hq):
+                kv = h // group
+                qa, ka, va, ga = q[b, h], k[b, kv], v[b, kv], g[b, h]
+                logits = (qa @ ka.T) * s if E else np.zeros((L, S))
+                if is_causal:
+                    logits = np.where(np.arange(S)[None, :] <= np.arange(L)[:, None], logits, -np.inf)
+                m = np.max(logits, axis=1, keepdims=True)
+                m = np.where(np.isfinite(m), m, 0.0)
+                p = np.exp(logits - m)
+                Z = p.sum(axis=1, keepdims=True)
+                P = np.where(Z > 0, p / np.where(Z > 0, Z, 1.0), 0.0)
+                out = P @ va
+                # relative error of each recomputed weight: the logit's, the
+                # forward logsumexp's (its budget), the subtraction and exp;
+                # the cast before P^T grad comes on top for dV
+                dl = abs(s) * gE * (np.abs(qa) @ np.abs(ka).T) if E else np.zeros((L, S))
+                dl = dl + 2 * _U32 * np.abs(np.where(np.isfinite(logits), logits, 0.0))
+                lse = m + np.log(np.where(Z > 0, Z, 1.0))
+                eta = dl + exp_rel + tol_l[b, h][:, None] + 2 * _U32 * (1 + np.abs(lse))
+                dP = ga @ va.T
+                adP = np.abs(ga) @ np.abs(va).T
+                D = (ga * out).sum(axis=1, keepdims=True)
+                # D from the forward's output in the input dtype (its budget
+                # includes the rounding) and the fp32 dot product
+                eD = (np.abs(ga) * tol_o[b, h]).sum(axis=1, keepdims=True)
+                eD = eD + gEv * (np.abs(ga) * np.abs(out)).sum(axis=1, keepdims=True)
+                dS = P * (dP - D)
+                edS = P * eta * np.abs(dP - D) + P * (gEv * adP + eD) + cast * np.abs(dS)
+                # dq = scale dS K
+                dq = s * (dS @ ka)
+                tdq[b, h] = abs(s) * (edS @ np.abs(ka) + gS * (np.abs(dS) @ np.abs(ka))) + ud * np.abs(dq)
+                # dk, dv summed over the group's query heads
+                adk[b, kv] += abs(s) * (np.abs(dS).T @ np.abs(qa))
+                tdk[b, kv] += abs(s) * (edS.T @ np.abs(qa))
+                dk_ex[b, kv] += s * (dS.T @ qa)
+                adv[b, kv] += P.T @ np.abs(ga)
+                tdv[b, kv] += ((P * (eta + cast)).T @ np.abs(ga))
+                dv_ex[b, kv] += P.T @ ga
+        tdk = tdk + gL * adk + ud * np.abs(dk_ex)
+        tdv = tdv + gL * adv + ud * np.abs(dv_ex)
+    return safety * tdq + 1e-30, safety * tdk + 1e-30, safety * tdv + 1e-30

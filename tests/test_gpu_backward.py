@@ -157,3 +157,32 @@ def test_backward_full_headline_sampled_heads():
                       g[b : b + 1, h : h + 1], is_causal=True)
         got = (dq[b : b + 1, h : h + 1], dk[b : b + 1, h : h + 1], dv[b : b + 1, h : h + 1])
         _check(got, ref, q.dtype, f"headline b={b} h={h}")
+
+
+BUDGET_CASES = [
+    # dtype, B, Hq, Hkv, L, S, E, causal   (16-bit E in {64, 96, 128}: tcgen05 kernels)
+    (torch.bfloat16, 1, 2, 2, 300, 300, 128, True),
+    (torch.float16, 1, 4, 2, 257, 130, 96, False),
+    (torch.bfloat16, 1, 2, 1, 129, 640, 64, True),
+    (torch.float16, 1, 2, 2, 90, 70, 32, False),      # general kernels
+    (torch.float32, 1, 2, 2, 80, 120, 40, True),
+]
+
+
+@pytest.mark.parametrize("case", BUDGET_CASES, ids=lambda c: "-".join(str(x) for x in c))
+def test_backward_within_the_error_budget(case):
+    """Every gradient element inside the per-element budget of the
+    FlashAttention backward (oracle/budget.py, backward_budget), which takes
+    the forward's own budget into the recomputed weights and D."""
+    from oracle.budget import backward_budget
+
+    dt, B, Hq, Hkv, L, S, E, causal = case
+    q, k, v = W.randn((B, Hq, L, E), 541, dt), W.randn((B, Hkv, S, E), 542, dt), W.randn((B, Hkv, S, E), 543, dt)
+    g = W.randn((B, Hq, L, E), 544, dt)
+    got = _run(q, k, v, g, is_causal=causal, enable_gqa=Hq != Hkv)
+    ref = ref_bwd(q, k, v, g, is_causal=causal, enable_gqa=Hq != Hkv)
+    name = {torch.float32: "float32", torch.float16: "float16", torch.bfloat16: "bfloat16"}[dt]
+    tols = backward_budget(q, k, v, g, dtype_name=name, is_causal=causal, enable_gqa=Hq != Hkv)
+    for gr, r, t, what in zip(got, ref, tols, ("dq", "dk", "dv")):
+        e = np.abs(gr.detach().double().cpu().numpy() - np.asarray(r))
+        assert (e <= t).all(), f"{what} outside the budget: max ratio {float((e / t).max()):.2f}"
