@@ -118,6 +118,12 @@ __device__ __forceinline__ bool wait(Bars* bars, uint64_t* bar, uint32_t parity)
   return ptx::mbar_wait(bar, parity, kTimeoutNs, &bars->abort);
 }
 
+// wait() taken by a whole warp, which agrees on the outcome.
+template <typename Bars>
+__device__ __forceinline__ bool wait_w(Bars* bars, uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, wait(bars, bar, parity));
+}
+
 __device__ __forceinline__ bool drain(uint64_t* bar, uint32_t parity) {
   const int never = 0;
   return ptx::mbar_wait(bar, parity, kTimeoutNs, &never);
@@ -138,12 +144,16 @@ __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
 
 // X = A B^T over a K dimension of D, both operands K-major in shared memory
 // (descriptor plus compile-time offsets), into tensor-memory columns at d.
-template <int D, int KK = 0>
+// kW: issued by a whole converged warp (ptx::mma_ss_off_w), else by one thread.
+template <int D, bool kW = false, int KK = 0>
 __device__ __forceinline__ void mma_kmajor(uint32_t d, uint64_t da, uint64_t db, uint32_t idesc) {
   if constexpr (KK < D / 16) {
     constexpr uint32_t off = ((KK / 4) * Tile<D>::BLOCK + (KK % 4) * 32) >> 4;
-    ptx::mma_ss_off<off, off>(d, da, db, idesc, KK > 0 ? 1u : 0u);
-    mma_kmajor<D, KK + 1>(d, da, db, idesc);
+    if constexpr (kW)
+      ptx::mma_ss_off_w<off, off>(d, da, db, idesc, KK > 0 ? 1u : 0u);
+    else
+      ptx::mma_ss_off<off, off>(d, da, db, idesc, KK > 0 ? 1u : 0u);
+    mma_kmajor<D, kW, KK + 1>(d, da, db, idesc);
   }
 }
 
@@ -152,12 +162,16 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d, uint64_t da, uint64_t db,
 // columns 0-63 are packed at a + [0, 32) and 64-127 at a + [64, 96) (each
 // warpgroup's own half of the columns it read).
 // KK in [KSTART, KEND) of the K = 128 products; the first one takes acc0.
-template <bool kSplit = false, int KSTART = 0, int KEND = BN / 16, int KK = KSTART>
+// kW as for mma_kmajor.
+template <bool kSplit = false, int KSTART = 0, int KEND = BN / 16, bool kW = false, int KK = KSTART>
 __device__ __forceinline__ void mma_tmem_a(uint32_t acc, uint32_t a, uint64_t db, uint32_t idesc, uint32_t acc0) {
   if constexpr (KK < KEND) {
     constexpr uint32_t col = kSplit ? (KK / 4) * 64 + (KK % 4) * 8 : KK * 8;
-    ptx::mma_ts_off<col, ((KK * 16 * 128) >> 4)>(acc, a, db, idesc, KK > KSTART ? 1u : acc0);
-    mma_tmem_a<kSplit, KSTART, KEND, KK + 1>(acc, a, db, idesc, acc0);
+    if constexpr (kW)
+      ptx::mma_ts_off_w<col, ((KK * 16 * 128) >> 4)>(acc, a, db, idesc, KK > KSTART ? 1u : acc0);
+    else
+      ptx::mma_ts_off<col, ((KK * 16 * 128) >> 4)>(acc, a, db, idesc, KK > KSTART ? 1u : acc0);
+    mma_tmem_a<kSplit, KSTART, KEND, kW, KK + 1>(acc, a, db, idesc, acc0);
   }
 }
 
@@ -299,8 +313,10 @@ bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         if (!drain(&bars->kfull[j % 3], (j / 3) & 1)) flag_error(bars, 12);
       for (int j = max(0, n - 2); j < n; ++j)
         if (!drain(&bars->vfull[j % 2], (j / 2) & 1)) flag_error(bars, 12);
-    } else if (warp == kWarpMma && lane == 0) {
+    } else if (warp == kWarpMma) {
       // ------------------------------------------------------------ MMA
+      // The whole warp runs this loop and one elected lane issues each
+      // tensor-core instruction.
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
       constexpr uint32_t idesc_s = ptx::idesc_f16(kBf16, BM, BN, false);
       constexpr uint32_t idesc_q = ptx::idesc_f16(kBf16, BM, D, true);
@@ -310,46 +326,46 @@ bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       const uint64_t dkmn = ptx::sdesc_sw128(ptx::smem_u32(smem + C::K_OFF), Tile<D>::BLOCK, 1024);
       const uint64_t dv_ = ptx::sdesc_sw128(ptx::smem_u32(smem + C::V_OFF), 16, 1024);
       constexpr uint64_t kStep = C::T >> 4;
-      bool ok = wait(bars, &bars->qg, 0) && wait(bars, &bars->kfull[0], 0);
+      bool ok = wait_w(bars, &bars->qg, 0) && wait_w(bars, &bars->kfull[0], 0);
       if (ok) {
         ptx::tc_fence_after();
-        mma_kmajor<D>(tmem, dq_, dk_, idesc_s);
-        ok = wait(bars, &bars->vfull[0], 0);
+        mma_kmajor<D, true>(tmem, dq_, dk_, idesc_s);
+        ok = wait_w(bars, &bars->vfull[0], 0);
       }
       if (ok) {
         ptx::tc_fence_after();
-        mma_kmajor<D>(tmem + 128, dg_, dv_, idesc_s);
-        ptx::mma_commit(&bars->sdp_ready);
-        ptx::mma_commit(&bars->vempty[0]);
+        mma_kmajor<D, true>(tmem + 128, dg_, dv_, idesc_s);
+        ptx::mma_commit_w(&bars->sdp_ready);
+        ptx::mma_commit_w(&bars->vempty[0]);
       }
       for (int j = 0; j < n && ok; ++j) {
         if (j + 1 < n) {
           // S and dP of the next key tile, once every thread has read this one's.
           const int ks = (j + 1) % 3, vs = (j + 1) % 2;
-          ok = wait(bars, &bars->sdp_free, j & 1) && wait(bars, &bars->kfull[ks], ((j + 1) / 3) & 1);
+          ok = wait_w(bars, &bars->sdp_free, j & 1) && wait_w(bars, &bars->kfull[ks], ((j + 1) / 3) & 1);
           if (!ok) break;
           ptx::tc_fence_after();
-          mma_kmajor<D>(tmem, dq_, dk_ + ks * kStep, idesc_s);
-          if (!wait(bars, &bars->vfull[vs], ((j + 1) / 2) & 1)) {
+          mma_kmajor<D, true>(tmem, dq_, dk_ + ks * kStep, idesc_s);
+          if (!wait_w(bars, &bars->vfull[vs], ((j + 1) / 2) & 1)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          mma_kmajor<D>(tmem + 128, dg_, dv_ + vs * kStep, idesc_s);
-          ptx::mma_commit(&bars->sdp_ready);
-          ptx::mma_commit(&bars->vempty[vs]);
+          mma_kmajor<D, true>(tmem + 128, dg_, dv_ + vs * kStep, idesc_s);
+          ptx::mma_commit_w(&bars->sdp_ready);
+          ptx::mma_commit_w(&bars->vempty[vs]);
         }
-        if (!wait(bars, &bars->ds_ready, j & 1)) {
+        if (!wait_w(bars, &bars->ds_ready, j & 1)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        mma_tmem_a(tmem + 384, tmem + 256, dkmn + (j % 3) * kStep, idesc_q, j > 0 ? 1u : 0u);
-        ptx::mma_commit(&bars->ds_free);
-        ptx::mma_commit(&bars->kempty[j % 3]);
+        mma_tmem_a<false, 0, BN / 16, true>(tmem + 384, tmem + 256, dkmn + (j % 3) * kStep, idesc_q, j > 0 ? 1u : 0u);
+        ptx::mma_commit_w(&bars->ds_free);
+        ptx::mma_commit_w(&bars->kempty[j % 3]);
       }
       if (!ok) flag_error(bars, 13);
-      ptx::mma_commit(&bars->done);
+      ptx::mma_commit_w(&bars->done);
       if (!drain(&bars->done, 0)) flag_error(bars, 14);
     }
   } else {
@@ -368,6 +384,7 @@ bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       Di = g.D[ridx];
     }
     const float sl = p.scale_log2;
+    const uint64_t sl2 = exp2poly::pk(sl, sl), nl2 = exp2poly::pk(-lse2, -lse2), nD2 = exp2poly::pk(-Di, -Di);
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       if (!__all_sync(0xffffffffu, wait(bars, &bars->sdp_ready, j & 1))) {
@@ -390,14 +407,27 @@ bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const int c0 = 2 * i, c1 = 2 * i + 1;
-        float p0 = exp2f_fast(__uint_as_float(s[c0 >> 5][c0 & 31]) * sl - lse2);
-        float p1 = exp2f_fast(__uint_as_float(s[c1 >> 5][c1 & 31]) * sl - lse2);
+        // Pairs in packed fp32x2 arithmetic; 1 pair of 4 takes 2^x on the FMA pipe.
+        const uint64_t x = exp2poly::ffma2(
+            exp2poly::pk(__uint_as_float(s[c0 >> 5][c0 & 31]), __uint_as_float(s[c1 >> 5][c1 & 31])), sl2, nl2);
+        float x0, x1, p0, p1;
+        exp2poly::upk(x, x0, x1);
+        if ((i & 3) == 3) {
+          exp2poly::exp2_pair(x0, x1, p0, p1);
+        } else {
+          p0 = exp2f_fast(x0);
+          p1 = exp2f_fast(x1);
+        }
         if (masked) {
           if (kv0 + c0 >= lim) p0 = 0.f;
           if (kv0 + c1 >= lim) p1 = 0.f;
         }
-        const float d0 = p0 * (__uint_as_float(dp[c0 >> 5][c0 & 31]) - Di);
-        const float d1 = p1 * (__uint_as_float(dp[c1 >> 5][c1 & 31]) - Di);
+        const uint64_t dd = exp2poly::fmul2(
+            exp2poly::pk(p0, p1),
+            exp2poly::fadd2(exp2poly::pk(__uint_as_float(dp[c0 >> 5][c0 & 31]), __uint_as_float(dp[c1 >> 5][c1 & 31])),
+                            nD2));
+        float d0, d1;
+        exp2poly::upk(dd, d0, d1);
         ds[i] = pack2<T>(d0, d1);
       }
       // dS has its own columns; the previous tile's dQ MMA must have read them.
@@ -525,8 +555,10 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!drain(&bars->kv, 0)) flag_error(bars, 22);
       for (int it = max(0, iters - 2); it < iters; ++it)
         if (!drain(&bars->qfull[it & 1], (it >> 1) & 1)) flag_error(bars, 22);
-    } else if (warp == kWarpMma && lane == 0) {
+    } else if (warp == kWarpMma) {
       // ------------------------------------------------------------ MMA
+      // The whole warp runs this loop and one elected lane issues each
+      // tensor-core instruction.
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
       // Query columns are handled in two halves (64 each), one per
       // elementwise warpgroup, so that one half's products overlap the other
@@ -547,11 +579,11 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // S^T and dP^T of query half hf of the tile in ring slot ns.
       auto scores = [&](int ns, int hf) {
         const uint64_t off = ns * kSlot + hf * kHalfRows;
-        mma_kmajor<D>(tmem + 64 * hf, dk_, dq_ + off, idesc_s);
-        mma_kmajor<D>(tmem + 128 + 64 * hf, dv_, dg_ + off, idesc_s);
-        ptx::mma_commit(&bars->sdp_ready[hf]);
+        mma_kmajor<D, true>(tmem + 64 * hf, dk_, dq_ + off, idesc_s);
+        mma_kmajor<D, true>(tmem + 128 + 64 * hf, dv_, dg_ + off, idesc_s);
+        ptx::mma_commit_w(&bars->sdp_ready[hf]);
       };
-      bool ok = iters == 0 || (wait(bars, &bars->kv, 0) && wait(bars, &bars->qfull[0], 0));
+      bool ok = iters == 0 || (wait_w(bars, &bars->kv, 0) && wait_w(bars, &bars->qfull[0], 0));
       if (ok && iters > 0) {
         ptx::tc_fence_after();
         scores(0, 0);
@@ -562,15 +594,15 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool next = it + 1 < iters;
         // Half 0: dV += P^T grad_i and dK += dS^T Q_i over query rows 0-63,
         // then (the next tile's Q_i and grad_i loaded) its next S^T, dP^T.
-        if (!wait(bars, &bars->pds_ready[0], it & 1)) {
+        if (!wait_w(bars, &bars->pds_ready[0], it & 1)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        mma_tmem_a<true, 0, 4>(tmem + 256, tmem, dgmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);
-        mma_tmem_a<true, 0, 4>(tmem + 384, tmem + 128, dqmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);
+        mma_tmem_a<true, 0, 4, true>(tmem + 256, tmem, dgmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);
+        mma_tmem_a<true, 0, 4, true>(tmem + 384, tmem + 128, dqmn + slot * kSlot, idesc_acc, it > 0 ? 1u : 0u);
         if (next) {
-          if (!wait(bars, &bars->qfull[ns], ((it + 1) >> 1) & 1)) {
+          if (!wait_w(bars, &bars->qfull[ns], ((it + 1) >> 1) & 1)) {
             ok = false;
             break;
           }
@@ -578,18 +610,18 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           scores(ns, 0);  // overwrites only half 0's columns
         }
         // Half 1.
-        if (!wait(bars, &bars->pds_ready[1], it & 1)) {
+        if (!wait_w(bars, &bars->pds_ready[1], it & 1)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        mma_tmem_a<true, 4, 8>(tmem + 256, tmem, dgmn + slot * kSlot, idesc_acc, 1u);
-        mma_tmem_a<true, 4, 8>(tmem + 384, tmem + 128, dqmn + slot * kSlot, idesc_acc, 1u);
-        ptx::mma_commit(&bars->qempty[slot]);
+        mma_tmem_a<true, 4, 8, true>(tmem + 256, tmem, dgmn + slot * kSlot, idesc_acc, 1u);
+        mma_tmem_a<true, 4, 8, true>(tmem + 384, tmem + 128, dqmn + slot * kSlot, idesc_acc, 1u);
+        ptx::mma_commit_w(&bars->qempty[slot]);
         if (next) scores(ns, 1);
       }
       if (!ok) flag_error(bars, 23);
-      ptx::mma_commit(&bars->done);
+      ptx::mma_commit_w(&bars->done);
       if (!drain(&bars->done, 0)) flag_error(bars, 24);
     }
   } else {
