@@ -174,28 +174,55 @@ __device__ __forceinline__ bool drain(uint64_t* bar, uint32_t parity) {
   return ptx::mbar_wait(bar, parity, kTimeoutNs, &never);
 }
 
+// kW: issued by the whole MMA warp (one elected lane issues each
+// instruction), else by one thread.
 // Lean issue: descriptors built once per CTA, operand addresses are the
 // descriptor plus compile-time offsets (address >> 4 in the low 14 bits never
 // carries inside shared memory).  S_i = Q_i K^T: A = Q_i (K-major), B = K
 // tile (K-major), D = tensor-memory columns [i*128, i*128+128).
-template <int D, int KK = 0>
+template <int D, bool kW, int KK = 0>
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint64_t dq_i, uint64_t dk, uint32_t idesc) {
   if constexpr (KK < D / 16) {
     constexpr uint32_t off = ((KK / 4) * Cfg<D>::BLOCK + (KK % 4) * 32) >> 4;
-    ptx::mma_ss_off<off, off>(tmem_s, dq_i, dk, idesc, KK > 0 ? 1u : 0u);
-    issue_qk<D, KK + 1>(tmem_s, dq_i, dk, idesc);
+    if constexpr (kW)
+      ptx::mma_ss_off_w<off, off>(tmem_s, dq_i, dk, idesc, KK > 0 ? 1u : 0u);
+    else
+      ptx::mma_ss_off<off, off>(tmem_s, dq_i, dk, idesc, KK > 0 ? 1u : 0u);
+    issue_qk<D, kW, KK + 1>(tmem_s, dq_i, dk, idesc);
   }
 }
 
 // O_i += P_i V: A = P_i from tensor memory (16-bit, packed over S_i), B = V
 // tile (MN-major).
-template <int KK = 0>
+template <bool kW, int KK = 0>
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t dv, uint32_t acc0,
                                          uint32_t idesc) {
   if constexpr (KK < BN / 16) {
-    ptx::mma_ts_off<KK * 8, ((KK * 16 * 128) >> 4)>(tmem_o, tmem_p, dv, idesc, KK > 0 ? 1u : acc0);
-    issue_pv<KK + 1>(tmem_o, tmem_p, dv, acc0, idesc);
+    if constexpr (kW)
+      ptx::mma_ts_off_w<KK * 8, ((KK * 16 * 128) >> 4)>(tmem_o, tmem_p, dv, idesc, KK > 0 ? 1u : acc0);
+    else
+      ptx::mma_ts_off<KK * 8, ((KK * 16 * 128) >> 4)>(tmem_o, tmem_p, dv, idesc, KK > 0 ? 1u : acc0);
+    issue_pv<kW, KK + 1>(tmem_o, tmem_p, dv, acc0, idesc);
   }
+}
+
+// Wait, outcome and commit of the MMA issuer in either form (kW: the whole
+// warp, every outcome made warp-uniform; else one thread).
+template <bool kW>
+__device__ __forceinline__ bool mma_uniform(bool ok) {
+  if constexpr (kW) return __all_sync(0xffffffffu, ok);
+  return ok;
+}
+template <bool kW>
+__device__ __forceinline__ bool mma_wait(Bars* bars, uint64_t* bar, uint32_t parity) {
+  return mma_uniform<kW>(wait(bars, bar, parity));
+}
+template <bool kW>
+__device__ __forceinline__ void mma_commit_as(uint64_t* bar) {
+  if constexpr (kW)
+    ptx::mma_commit_w(bar);
+  else
+    ptx::mma_commit(bar);
 }
 
 // All 128 columns of S (four 32-column blocks) with one instruction.
@@ -386,6 +413,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   Bars* bars = reinterpret_cast<Bars*>(smem + C::BAR_OFF);
 
   const bool causal = (p.mask == SDPA_MASK_CAUSAL) || (p.mask == SDPA_MASK_BLOCK_DIAG_CAUSAL);
+  constexpr bool kWI = D == 128;  // MMA issue by the whole warp
   const int bx = kVarlen ? p.n_seqs : p.B;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -485,8 +513,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!drain(&bars->full[v % C::NS], (v / C::NS) & 1)) flag_error(bars, 2);
       for (int sub = 0; sub < NSUB; ++sub)
         if (nq[sub] > 0 && !drain(&bars->q[sub], (nq[sub] - 1) & 1)) flag_error(bars, 2);
-    } else if (warp == kWarpMma && lane == 0) {
+    } else if (warp == kWarpMma && (kWI || lane == 0)) {
       // ---------------------------------------------------------- MMA issuer
+      // For E = 128 the whole warp runs this loop (every decision
+      // warp-uniform) and one elected lane issues each tensor-core
+      // instruction and commit, which keeps the issue up with the tensor
+      // pipe while the softmax warps load the sub-partitions (measured: 1 %
+      // faster at E = 128, 2-3 % slower at E = 64 and 96, where one thread
+      // issues).
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
       constexpr uint32_t idesc_qk = ptx::idesc_f16(kBf16, BM, BN, false);
       constexpr uint32_t idesc_pv = ptx::idesc_f16(kBf16, BM, D, true);
@@ -498,26 +532,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       int t = 0, k = 0;  // ring position of the unit's K_0; units done
       int tile0 = 0, tile1 = 0;  // key tiles whose P each sub-tile has handed over
       int idx = -1;
-      bool ok = read_unit(bars, 0, idx);
-      if (ok) ptx::mbar_arrive(&bars->unit_empty[0]);
+      bool ok = mma_uniform<kWI>(read_unit(bars, 0, idx));
+      if (ok && (!kWI || lane == 0)) ptx::mbar_arrive(&bars->unit_empty[0]);
       bool have = ok && idx >= 0;
       Unit u;
       if (have) {
         unit_at<kVarlen>(p, idx, bx, mblocks, causal, u);
         // Scores of the first unit's first key tile.
-        ok = wait(bars, &bars->full[0], 0);
+        ok = mma_wait<kWI>(bars, &bars->full[0], 0);
 #pragma unroll 1
         for (int sub = 0; sub < NSUB && ok; ++sub) {
-          if (!wait(bars, &bars->q[sub], 0)) {
+          if (!mma_wait<kWI>(bars, &bars->q[sub], 0)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          issue_qk<D>(tmem + sub * 128, dq + sub * kSubStep, dk0, idesc_qk);
-          ptx::mma_commit(&bars->s[sub]);
-          if (u.n_kv == 1) ptx::mma_commit(&bars->q_free[sub]);
+          issue_qk<D, kWI>(tmem + sub * 128, dq + sub * kSubStep, dk0, idesc_qk);
+          mma_commit_as<kWI>(&bars->s[sub]);
+          if (u.n_kv == 1) mma_commit_as<kWI>(&bars->q_free[sub]);
         }
-        if (ok) ptx::mma_commit(&bars->empty[0]);
+        if (ok) mma_commit_as<kWI>(&bars->empty[0]);
       }
       while (have && ok) {
         const int n = u.n_kv;
@@ -530,76 +564,76 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const uint32_t acc = j > 0 ? 1u : 0u;
           // The first PV of a unit overwrites O: its P is written only after
           // the softmax warpgroup has read the previous unit's O out.
-          ok = wait(bars, &bars->full[vslot], (vt / C::NS) & 1) && wait(bars, &bars->p[0], tile0 & 1);
+          ok = mma_wait<kWI>(bars, &bars->full[vslot], (vt / C::NS) & 1) && mma_wait<kWI>(bars, &bars->p[0], tile0 & 1);
           if (!ok) break;
           ++tile0;
           ptx::tc_fence_after();
-          issue_pv(tmem + 256, tmem, dv, acc, idesc_pv);
-          if (!wait(bars, &bars->full[kslot], (kt / C::NS) & 1)) {
+          issue_pv<kWI>(tmem + 256, tmem, dv, acc, idesc_pv);
+          if (!mma_wait<kWI>(bars, &bars->full[kslot], (kt / C::NS) & 1)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          issue_qk<D>(tmem, dq, dk, idesc_qk);
-          ptx::mma_commit(&bars->s[0]);
-          if (j + 2 == n) ptx::mma_commit(&bars->q_free[0]);  // last scores of the unit
-          if (!wait(bars, &bars->p[1], tile1 & 1)) {
+          issue_qk<D, kWI>(tmem, dq, dk, idesc_qk);
+          mma_commit_as<kWI>(&bars->s[0]);
+          if (j + 2 == n) mma_commit_as<kWI>(&bars->q_free[0]);  // last scores of the unit
+          if (!mma_wait<kWI>(bars, &bars->p[1], tile1 & 1)) {
             ok = false;
             break;
           }
           ++tile1;
           ptx::tc_fence_after();
-          issue_pv(tmem + 384, tmem + 128, dv, acc, idesc_pv);
-          issue_qk<D>(tmem + 128, dq + kSubStep, dk, idesc_qk);
-          ptx::mma_commit(&bars->s[1]);
-          if (j + 2 == n) ptx::mma_commit(&bars->q_free[1]);
-          ptx::mma_commit(&bars->empty[vslot]);
-          ptx::mma_commit(&bars->empty[kslot]);
+          issue_pv<kWI>(tmem + 384, tmem + 128, dv, acc, idesc_pv);
+          issue_qk<D, kWI>(tmem + 128, dq + kSubStep, dk, idesc_qk);
+          mma_commit_as<kWI>(&bars->s[1]);
+          if (j + 2 == n) mma_commit_as<kWI>(&bars->q_free[1]);
+          mma_commit_as<kWI>(&bars->empty[vslot]);
+          mma_commit_as<kWI>(&bars->empty[kslot]);
         }
         if (!ok) break;
         // Last key tile: PV_i(n-1), then the next unit's first scores.
         const int vt = t + 2 * n - 1, vslot = vt % C::NS;
         const int kt = t + 2 * n, kslot = kt % C::NS;  // the next unit's K_0
         int nidx = -1;
-        ok = wait(bars, &bars->full[vslot], (vt / C::NS) & 1) && read_unit(bars, k + 1, nidx);
+        ok = mma_wait<kWI>(bars, &bars->full[vslot], (vt / C::NS) & 1) && mma_uniform<kWI>(read_unit(bars, k + 1, nidx));
         if (!ok) break;
-        ptx::mbar_arrive(&bars->unit_empty[(k + 1) % kUnitRing]);
+        if (!kWI || lane == 0) ptx::mbar_arrive(&bars->unit_empty[(k + 1) % kUnitRing]);
         Unit nx;
         const bool nx_have = nidx >= 0;
         if (nx_have) unit_at<kVarlen>(p, nidx, bx, mblocks, causal, nx);
 #pragma unroll 1
         for (int sub = 0; sub < NSUB; ++sub) {
-          if (!wait(bars, &bars->p[sub], (sub ? tile1 : tile0) & 1)) {
+          if (!mma_wait<kWI>(bars, &bars->p[sub], (sub ? tile1 : tile0) & 1)) {
             ok = false;
             break;
           }
           if (sub) ++tile1;
           else ++tile0;
           ptx::tc_fence_after();
-          issue_pv(tmem + 256 + sub * 128, tmem + sub * 128, dv0 + vslot * kSlotStep, n > 1 ? 1u : 0u, idesc_pv);
-          ptx::mma_commit(&bars->o[sub]);  // this sub-tile's output is final
+          issue_pv<kWI>(tmem + 256 + sub * 128, tmem + sub * 128, dv0 + vslot * kSlotStep, n > 1 ? 1u : 0u, idesc_pv);
+          mma_commit_as<kWI>(&bars->o[sub]);  // this sub-tile's output is final
           if (!nx_have) continue;
-          if ((sub == 0 && !wait(bars, &bars->full[kslot], (kt / C::NS) & 1)) ||
-              !wait(bars, &bars->q[sub], (k + 1) & 1)) {
+          if ((sub == 0 && !mma_wait<kWI>(bars, &bars->full[kslot], (kt / C::NS) & 1)) ||
+              !mma_wait<kWI>(bars, &bars->q[sub], (k + 1) & 1)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          issue_qk<D>(tmem + sub * 128, dq + sub * kSubStep, dk0 + kslot * kSlotStep, idesc_qk);
-          ptx::mma_commit(&bars->s[sub]);
-          if (nx.n_kv == 1) ptx::mma_commit(&bars->q_free[sub]);  // the next unit's last scores
+          issue_qk<D, kWI>(tmem + sub * 128, dq + sub * kSubStep, dk0 + kslot * kSlotStep, idesc_qk);
+          mma_commit_as<kWI>(&bars->s[sub]);
+          if (nx.n_kv == 1) mma_commit_as<kWI>(&bars->q_free[sub]);  // the next unit's last scores
         }
         if (!ok) break;
-        ptx::mma_commit(&bars->empty[vslot]);
+        mma_commit_as<kWI>(&bars->empty[vslot]);
         if (!nx_have) break;
-        ptx::mma_commit(&bars->empty[kslot]);
+        mma_commit_as<kWI>(&bars->empty[kslot]);
         t += 2 * n;
         ++k;
         u = nx;
       }
       if (!ok) flag_error(bars, 3);
       // Every MMA issued above completes before tensor memory is freed.
-      ptx::mma_commit(&bars->done);
+      mma_commit_as<kWI>(&bars->done);
       if (!drain(&bars->done, 0)) flag_error(bars, 4);
     }
   } else {
