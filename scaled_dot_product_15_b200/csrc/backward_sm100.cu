@@ -34,6 +34,7 @@
 // an error word (sdpa_take_device_error reports it), stops its other roles, drains what it
 // issued and returns.
 #include <algorithm>
+#include <type_traits>
 
 #include "backward.cuh"
 #include "exp2_poly.cuh"
@@ -403,33 +404,37 @@ bwd_dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       const int kv0 = j * BN + 64 * w;
       const bool masked = !row_ok || kv0 + 64 > Sk || (causal && kv0 + 63 > row0);  // warp-uniform
       const int lim = !row_ok ? 0 : (causal ? min(Sk, rg + 1) : Sk);  // keys [0, lim) are kept
+      const int cmax = lim - kv0;  // this tile's columns c < cmax are kept
       uint32_t ds[32];
+      // Two straight-line copies of the loop (masked is warp-uniform): a mask
+      // test between the pairs would split the unrolled loop into small blocks.
+      auto form = [&](auto kMasked) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int c0 = 2 * i, c1 = 2 * i + 1;
-        // Pairs in packed fp32x2 arithmetic; 1 pair of 4 takes 2^x on the FMA pipe.
-        const uint64_t x = exp2poly::ffma2(
-            exp2poly::pk(__uint_as_float(s[c0 >> 5][c0 & 31]), __uint_as_float(s[c1 >> 5][c1 & 31])), sl2, nl2);
-        float x0, x1, p0, p1;
-        exp2poly::upk(x, x0, x1);
-        if ((i & 3) == 3) {
-          exp2poly::exp2_pair(x0, x1, p0, p1);
-        } else {
-          p0 = exp2f_fast(x0);
-          p1 = exp2f_fast(x1);
+        for (int i = 0; i < 32; ++i) {
+          const int c0 = 2 * i, c1 = 2 * i + 1;
+          // Pairs in packed fp32x2 arithmetic.
+          const uint64_t x = exp2poly::ffma2(
+              exp2poly::pk(__uint_as_float(s[c0 >> 5][c0 & 31]), __uint_as_float(s[c1 >> 5][c1 & 31])), sl2, nl2);
+          float x0, x1;
+          exp2poly::upk(x, x0, x1);
+          float p0 = exp2f_fast(x0), p1 = exp2f_fast(x1);
+          if constexpr (decltype(kMasked)::value) {
+            p0 = c0 < cmax ? p0 : 0.f;
+            p1 = c1 < cmax ? p1 : 0.f;
+          }
+          const uint64_t dd = exp2poly::fmul2(
+              exp2poly::pk(p0, p1),
+              exp2poly::fadd2(
+                  exp2poly::pk(__uint_as_float(dp[c0 >> 5][c0 & 31]), __uint_as_float(dp[c1 >> 5][c1 & 31])), nD2));
+          float d0, d1;
+          exp2poly::upk(dd, d0, d1);
+          ds[i] = pack2<T>(d0, d1);
         }
-        if (masked) {
-          if (kv0 + c0 >= lim) p0 = 0.f;
-          if (kv0 + c1 >= lim) p1 = 0.f;
-        }
-        const uint64_t dd = exp2poly::fmul2(
-            exp2poly::pk(p0, p1),
-            exp2poly::fadd2(exp2poly::pk(__uint_as_float(dp[c0 >> 5][c0 & 31]), __uint_as_float(dp[c1 >> 5][c1 & 31])),
-                            nD2));
-        float d0, d1;
-        exp2poly::upk(dd, d0, d1);
-        ds[i] = pack2<T>(d0, d1);
-      }
+      };
+      if (masked)
+        form(std::true_type{});
+      else
+        form(std::false_type{});
       // dS has its own columns; the previous tile's dQ MMA must have read them.
       if (j > 0 && !__all_sync(0xffffffffu, wait(bars, &bars->ds_free, (j - 1) & 1))) {
         ok = false;
@@ -668,42 +673,47 @@ bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ok = false;
         break;
       }
+      // Query columns c < cmin of this thread's key row are masked out (all
+      // of them for a key past the end; under a causal mask the columns of
+      // queries before the key).  Columns of query rows past the end have
+      // lse = +inf staged, so their weights are 2^-inf = 0 already.
       const int qc0 = q0 + 64 * w;
-      const bool masked = qc0 + 64 > Lq || kj >= Sk || (causal && kj > qc0);  // per thread
+      const int cmin = kj >= Sk ? 64 : (causal ? kj - qc0 : 0);
+      // Two straight-line copies of the loop, chosen per warp: a mask test
+      // between the pairs would split the unrolled loop into small blocks.
+      auto form = [&](auto kMasked) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pp[16], dsp[16];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pp[16], dsp[16];
 #pragma unroll
-        for (int qd = 0; qd < 8; ++qd) {  // 4 query columns at a time
-          const int c = 32 * half + 4 * qd;
-          const float4 l4 = *reinterpret_cast<const float4*>(lv + c);
-          const float4 d4 = *reinterpret_cast<const float4*>(lv + 64 + c);
-          const float ls[4] = {l4.x, l4.y, l4.z, l4.w}, ds[4] = {d4.x, d4.y, d4.z, d4.w};
+          for (int qd = 0; qd < 8; ++qd) {  // 4 query columns at a time
+            const int c = 32 * half + 4 * qd;
+            const float4 l4 = *reinterpret_cast<const float4*>(lv + c);
+            const float4 d4 = *reinterpret_cast<const float4*>(lv + 64 + c);
+            const float ls[4] = {l4.x, l4.y, l4.z, l4.w}, ds[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-          for (int pr = 0; pr < 2; ++pr) {
-            const int c0 = c + 2 * pr, c1 = c0 + 1;
-            const float x0 = __uint_as_float(s[c0 >> 5][c0 & 31]) * sl - ls[2 * pr];
-            const float x1 = __uint_as_float(s[c1 >> 5][c1 & 31]) * sl - ls[2 * pr + 1];
-            float p0, p1;
-            if (pr == 1 && (qd & 1)) {
-              exp2poly::exp2_pair(x0, x1, p0, p1);  // 1 of 4 pairs on the FMA pipe
-            } else {
-              p0 = exp2f_fast(x0);
-              p1 = exp2f_fast(x1);
+            for (int pr = 0; pr < 2; ++pr) {
+              const int c0 = c + 2 * pr, c1 = c0 + 1;
+              float p0 = exp2f_fast(__uint_as_float(s[c0 >> 5][c0 & 31]) * sl - ls[2 * pr]);
+              float p1 = exp2f_fast(__uint_as_float(s[c1 >> 5][c1 & 31]) * sl - ls[2 * pr + 1]);
+              if constexpr (decltype(kMasked)::value) {
+                p0 = c0 >= cmin ? p0 : 0.f;
+                p1 = c1 >= cmin ? p1 : 0.f;
+              }
+              const float d0 = p0 * (__uint_as_float(dp[c0 >> 5][c0 & 31]) - ds[2 * pr]);
+              const float d1 = p1 * (__uint_as_float(dp[c1 >> 5][c1 & 31]) - ds[2 * pr + 1]);
+              pp[2 * qd + pr] = pack2<T>(p0, p1);
+              dsp[2 * qd + pr] = pack2<T>(d0, d1);
             }
-            if (masked) {
-              if (kj >= Sk || (causal && kj > q0 + 64 * w + c0)) p0 = 0.f;
-              if (kj >= Sk || (causal && kj > q0 + 64 * w + c1)) p1 = 0.f;
-            }
-            const float d0 = p0 * (__uint_as_float(dp[c0 >> 5][c0 & 31]) - ds[2 * pr]);
-            const float d1 = p1 * (__uint_as_float(dp[c1 >> 5][c1 & 31]) - ds[2 * pr + 1]);
-            pp[2 * qd + pr] = pack2<T>(p0, p1);
-            dsp[2 * qd + pr] = pack2<T>(d0, d1);
           }
+          tmem_st16(tmem + lane_off + 64 * w + 16 * half, pp);
+          tmem_st16(tmem + lane_off + 128 + 64 * w + 16 * half, dsp);
         }
-        tmem_st16(tmem + lane_off + 64 * w + 16 * half, pp);
-        tmem_st16(tmem + lane_off + 128 + 64 * w + 16 * half, dsp);
-      }
+      };
+      if (__any_sync(0xffffffffu, cmin > 0))
+        form(std::true_type{});
+      else
+        form(std::false_type{});
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars->pds_ready[w]);
