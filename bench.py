@@ -59,7 +59,7 @@ KERNEL_SOURCES = {
     "simt": ["simt.cu", "common.cuh"],
     "backward_simt": ["backward_simt.cu", "backward.cuh", "common.cuh"],
     "backward_tcgen05": ["backward_sm100.cu", "backward_simt.cu", "backward.cuh", "tma_host.cuh", "sm100_ptx.cuh",
-                         "common.cuh"],
+                         "exp2_poly.cuh", "common.cuh"],
 }
 
 
