@@ -21,7 +21,8 @@
 //               unit's last scores of that sub-tile have read it), V_0, K_1,
 //               V_1, ... as 128-key tiles through a ring of shared-memory
 //               slots (128-byte swizzle, 64-column boxes).
-//   warp 8      MMA issuer (one thread): S_i = Q_i K_j^T with both operands in
+//   warp 8      MMA issuer (one thread; at E = 128 the whole warp, one elected
+//               lane issuing): S_i = Q_i K_j^T with both operands in
 //               shared memory, O_i += P_i V_j with P_i read from tensor memory;
 //               fp32 accumulators in tensor memory (S0 | S1 | O0 | O1 = 512
 //               columns).  Sub-tiles interleave (PV0, S0 next, PV1, S1 next) so
@@ -41,7 +42,9 @@
 //               dtype straight from tensor memory to global memory and
 //               lse = (m + log2 l) * ln 2, while the next unit's first scores
 //               are already being computed.
-// Causal attention visits only key tiles at or left of the diagonal; packed
+// Causal attention visits only key tiles at or left of the diagonal, per
+// sub-tile: the last key tile of a 256-row unit lies wholly above sub-tile 0's
+// rows, so sub-tile 0 skips its scores, softmax and PV.  Packed
 // variable-length batches index tiles from each segment's first token.
 //
 // Every wait on an mbarrier is bounded (2 s); on a timeout the kernel records
@@ -127,7 +130,10 @@ static_assert(sizeof(Bars) <= 512, "barrier block");
 
 // A work unit: 256 query rows of one (batch or segment, head).
 struct Unit {
-  int h, b, seq0, Lq, Sk, row0, n_kv;
+  int h, b, seq0, Lq, Sk, row0;
+  int n_kv;  // key tiles of the unit (sub-tile 1's)
+  int n0;    // key tiles of sub-tile 0: n_kv, or n_kv - 1 under a causal mask
+             // when the last tile lies wholly above sub-tile 0's rows
 };
 
 template <typename T>
@@ -337,9 +343,13 @@ __device__ __forceinline__ bool unit_at(const Params& p, int idx, int bx, int mb
   }
   u.row0 = mb * (NSUB * BM);
   if (u.row0 >= u.Lq || u.Sk <= 0) return false;
-  int n = (u.Sk + BN - 1) / BN;
-  if (causal) n = min(n, (min(u.row0 + NSUB * BM, u.Lq) - 1) / BN + 1);
+  int n = (u.Sk + BN - 1) / BN, n0 = n;
+  if (causal) {
+    n = min(n, (min(u.row0 + NSUB * BM, u.Lq) - 1) / BN + 1);
+    n0 = min(n, (min(u.row0 + BM, u.Lq) - 1) / BN + 1);  // n - 1 or n
+  }
   u.n_kv = n;
+  u.n0 = n0;
   return true;
 }
 
@@ -549,7 +559,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           ptx::tc_fence_after();
           issue_qk<D, kWI>(tmem + sub * 128, dq + sub * kSubStep, dk0, idesc_qk);
           mma_commit_as<kWI>(&bars->s[sub]);
-          if (u.n_kv == 1) mma_commit_as<kWI>(&bars->q_free[sub]);
+          if ((sub ? u.n_kv : u.n0) == 1) mma_commit_as<kWI>(&bars->q_free[sub]);
         }
         if (ok) mma_commit_as<kWI>(&bars->empty[0]);
       }
@@ -573,10 +583,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             ok = false;
             break;
           }
-          ptx::tc_fence_after();
-          issue_qk<D, kWI>(tmem, dq, dk, idesc_qk);
-          mma_commit_as<kWI>(&bars->s[0]);
-          if (j + 2 == n) mma_commit_as<kWI>(&bars->q_free[0]);  // last scores of the unit
+          if (j + 1 < u.n0) {  // sub-tile 0 may skip the unit's last key tile
+            ptx::tc_fence_after();
+            issue_qk<D, kWI>(tmem, dq, dk, idesc_qk);
+            mma_commit_as<kWI>(&bars->s[0]);
+            if (j + 2 == u.n0) mma_commit_as<kWI>(&bars->q_free[0]);  // its last scores of the unit
+          }
           if (!mma_wait<kWI>(bars, &bars->p[1], tile1 & 1)) {
             ok = false;
             break;
@@ -591,7 +603,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           mma_commit_as<kWI>(&bars->empty[kslot]);
         }
         if (!ok) break;
-        // Last key tile: PV_i(n-1), then the next unit's first scores.
+        // Last key tile: PV_i(n-1) (sub-tile 0's last PV already ran above
+        // when it skips this tile), then the next unit's first scores.
         const int vt = t + 2 * n - 1, vslot = vt % C::NS;
         const int kt = t + 2 * n, kslot = kt % C::NS;  // the next unit's K_0
         int nidx = -1;
@@ -603,14 +616,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (nx_have) unit_at<kVarlen>(p, nidx, bx, mblocks, causal, nx);
 #pragma unroll 1
         for (int sub = 0; sub < NSUB; ++sub) {
-          if (!mma_wait<kWI>(bars, &bars->p[sub], (sub ? tile1 : tile0) & 1)) {
-            ok = false;
-            break;
+          if (sub == 1 || u.n0 == n) {
+            if (!mma_wait<kWI>(bars, &bars->p[sub], (sub ? tile1 : tile0) & 1)) {
+              ok = false;
+              break;
+            }
+            if (sub) ++tile1;
+            else ++tile0;
+            ptx::tc_fence_after();
+            issue_pv<kWI>(tmem + 256 + sub * 128, tmem + sub * 128, dv0 + vslot * kSlotStep, n > 1 ? 1u : 0u,
+                          idesc_pv);
           }
-          if (sub) ++tile1;
-          else ++tile0;
-          ptx::tc_fence_after();
-          issue_pv<kWI>(tmem + 256 + sub * 128, tmem + sub * 128, dv0 + vslot * kSlotStep, n > 1 ? 1u : 0u, idesc_pv);
           mma_commit_as<kWI>(&bars->o[sub]);  // this sub-tile's output is final
           if (!nx_have) continue;
           if ((sub == 0 && !mma_wait<kWI>(bars, &bars->full[kslot], (kt / C::NS) & 1)) ||
@@ -621,7 +637,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           ptx::tc_fence_after();
           issue_qk<D, kWI>(tmem + sub * 128, dq + sub * kSubStep, dk0 + kslot * kSlotStep, idesc_qk);
           mma_commit_as<kWI>(&bars->s[sub]);
-          if (nx.n_kv == 1) mma_commit_as<kWI>(&bars->q_free[sub]);  // the next unit's last scores
+          if ((sub ? nx.n_kv : nx.n0) == 1) mma_commit_as<kWI>(&bars->q_free[sub]);  // the next unit's last scores
         }
         if (!ok) break;
         mma_commit_as<kWI>(&bars->empty[vslot]);
@@ -659,7 +675,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int row_lo = u.row0 + sub * BM;
       const int r = row_lo + rin;  // query row within the sequence
       float m_run = -INFINITY, l_run = 0.f;
-      for (int j = 0; j < u.n_kv; ++j, ++tile) {
+      const int n_sub = sub ? u.n_kv : u.n0;
+      for (int j = 0; j < n_sub; ++j, ++tile) {
         // Every wait's outcome is made warp-uniform, so a timeout can never
         // leave part of a warp inside a warp-collective tcgen05 instruction.
         if (!__all_sync(0xffffffffu, wait(bars, &bars->s[sub], tile & 1))) {

@@ -18,6 +18,11 @@ against a model of the hardware:
   once every earlier MMA has executed;
 * TMA loads land at arbitrary later times.
 
+A unit is given as its number of key tiles n, or as (n0, n) when sub-tile 0
+needs only its first n0 = n - 1 tiles (under a causal mask the last key tile
+of a 256-row block lies wholly above sub-tile 0's rows, and the kernel skips
+that tile's scores, softmax and PV for it).
+
 Random interleavings are explored for several unit lists.  Besides deadlock and
 aliasing, every buffer (Q_i, the key/value ring slots, S/P and O in tensor
 memory) carries the tag of what
@@ -65,7 +70,9 @@ class Model:
     READERS = 3  # MMA, softmax 0, softmax 1
 
     def __init__(self, units, ns, rng):
-        self.units, self.ns, self.rng = units, ns, rng
+        self.ntiles = [u if isinstance(u, tuple) else (u, u) for u in units]
+        self.units = [u[1] for u in self.ntiles]
+        self.ns, self.rng = ns, rng
         B = Bar
         self.q = [B(f"q{a}", 1) for a in range(2)]
         self.q_free = [B(f"q_free{a}", 1) for a in range(2)]
@@ -85,6 +92,10 @@ class Model:
         self.s_exec = [(-1, 0), (-1, 0)]  # last (unit, tile) S MMA executed per sub-tile
         self.pipe = []                   # in-order tensor pipe
         self.tma = []                    # (slot, tag) loads in flight
+
+    def nsub(self, k, sub):
+        """Key tiles sub-tile `sub` of unit k takes."""
+        return self.ntiles[k][0] if sub == 0 else self.ntiles[k][1]
 
     # -- hardware -------------------------------------------------------
     def check_wait(self, bar, parity, phase):
@@ -167,7 +178,7 @@ class Model:
                         for sub in range(2):
                             if nq[sub] > 0:
                                 yield ("wait", self.q_free[sub], (nq[sub] - 1) & 1, nq[sub] - 1)
-                                if self.s_exec[sub] < (k - 1, self.units[k - 1] - 1):
+                                if self.s_exec[sub] < (k - 1, self.nsub(k - 1, sub) - 1):
                                     raise ProtocolError(f"Q{sub} of unit {k} loaded under pending score MMAs of unit {k - 1}")
                             self.qbuf[sub] = ("loading",)
                             self.tma.append((f"q{sub}", ("Q", k)))
@@ -178,6 +189,8 @@ class Model:
                     if old is not None:  # nothing may still need the old tile
                         kind, ok, oj = old
                         for sub in range(2):
+                            if oj >= self.nsub(ok, sub):
+                                continue  # a tile this sub-tile skips
                             if kind == "K" and self.s_exec[sub] < (ok, oj):
                                 raise ProtocolError(f"K({ok},{oj}) slot refilled before S{sub} read it")
                             if kind == "V" and (self.obuf[sub] is None or self.obuf[sub] < (ok, oj + 1)):
@@ -197,7 +210,7 @@ class Model:
             yield ("wait", self.q[sub], 0, 0)
             self.pipe.append(("qk", sub, 0, cur, 0))
             self.pipe.append(("commit", self.s[sub]))
-            if self.units[cur] == 1:
+            if self.nsub(cur, sub) == 1:
                 self.pipe.append(("commit", self.q_free[sub]))
         self.pipe.append(("commit", self.empty[0]))
         while True:
@@ -208,15 +221,17 @@ class Model:
                 vslot, kslot = vt % ns, kt % ns
                 yield ("wait", self.full[vslot], (vt // ns) & 1, vt // ns)
                 for sub in range(2):
+                    nsub = self.nsub(cur, sub)
                     yield ("wait", self.p[sub], tile[sub] & 1, tile[sub])
                     tile[sub] += 1
                     self.pipe.append(("pv", sub, vslot, cur, j))
                     if sub == 0:
                         yield ("wait", self.full[kslot], (kt // ns) & 1, kt // ns)
-                    self.pipe.append(("qk", sub, kslot, cur, j + 1))
-                    self.pipe.append(("commit", self.s[sub]))
-                    if j + 2 == n:
-                        self.pipe.append(("commit", self.q_free[sub]))
+                    if j + 1 < nsub:
+                        self.pipe.append(("qk", sub, kslot, cur, j + 1))
+                        self.pipe.append(("commit", self.s[sub]))
+                        if j + 2 == nsub:
+                            self.pipe.append(("commit", self.q_free[sub]))
                 self.pipe.append(("commit", self.empty[vslot]))
                 self.pipe.append(("commit", self.empty[kslot]))
             # last key tile, then the next unit's first scores
@@ -225,9 +240,10 @@ class Model:
             yield ("wait", self.full[vslot], (vt // ns) & 1, vt // ns)
             nxt = yield from self.read_unit(k + 1)
             for sub in range(2):
-                yield ("wait", self.p[sub], tile[sub] & 1, tile[sub])
-                tile[sub] += 1
-                self.pipe.append(("pv", sub, vslot, cur, n - 1))
+                if self.nsub(cur, sub) == n:  # else its last PV ran in the steady loop
+                    yield ("wait", self.p[sub], tile[sub] & 1, tile[sub])
+                    tile[sub] += 1
+                    self.pipe.append(("pv", sub, vslot, cur, n - 1))
                 self.pipe.append(("commit", self.o[sub]))
                 if nxt < 0:
                     continue
@@ -236,7 +252,7 @@ class Model:
                 yield ("wait", self.q[sub], (k + 1) & 1, k + 1)
                 self.pipe.append(("qk", sub, kslot, nxt, 0))
                 self.pipe.append(("commit", self.s[sub]))
-                if self.units[nxt] == 1:
+                if self.nsub(nxt, sub) == 1:
                     self.pipe.append(("commit", self.q_free[sub]))
             self.pipe.append(("commit", self.empty[vslot]))
             if nxt < 0:
@@ -252,7 +268,7 @@ class Model:
             cur = yield from self.read_unit(k)
             if cur < 0:
                 return
-            n = self.units[cur]
+            n = self.nsub(cur, sub)
             for j in range(n):
                 yield ("wait", self.s[sub], tile & 1, tile)
                 if self.sbuf[sub] != ("S", cur, j):
@@ -303,14 +319,17 @@ class Model:
         raise ProtocolError("did not finish")
 
 
-UNIT_LISTS = [[1], [2], [3], [5], [16], [33], [1, 1, 1], [3, 1, 2], [5, 5], [1, 4, 2, 6, 1], [16, 8, 2], [2, 2, 2, 2, 2]]
+UNIT_LISTS = [[1], [2], [3], [5], [16], [33], [1, 1, 1], [3, 1, 2], [5, 5], [1, 4, 2, 6, 1], [16, 8, 2], [2, 2, 2, 2, 2],
+              # sub-tile 0 skipping the last key tile (causal row blocks)
+              [(1, 2)], [(15, 16), (7, 8), (1, 2)], [(1, 2), (1, 2), (1, 2)], [(3, 4), 2, (1, 2), 1, (5, 6)],
+              [1, (1, 2), (2, 3), 3]]
 
 
-@pytest.mark.parametrize("units", UNIT_LISTS, ids=lambda u: "-".join(map(str, u)))
+@pytest.mark.parametrize("units", UNIT_LISTS, ids=lambda u: "-".join(map(str, u)).replace(" ", ""))
 @pytest.mark.parametrize("ns", [4, 8])
 def test_protocol_random_interleavings(units, ns):
     for seed in range(30):
-        Model(units, ns, random.Random(seed * 1000 + sum(units) * 37 + ns)).run()
+        Model(units, ns, random.Random(seed * 1000 + sum(u if isinstance(u, int) else u[1] for u in units) * 37 + ns)).run()
 
 
 def _caught(cls, units=(3, 1, 4, 2), ns=4):
@@ -393,3 +412,17 @@ def test_model_catches_q_released_too_early():
 
     assert _caught(EarlyQ)
 
+
+
+def test_model_catches_a_skipped_tile_still_waited_for():
+    """Sub-tile 0's softmax taking all n tiles of a unit whose last tile the
+    MMA issuer skips for it waits on scores that never come."""
+
+    class Mismatch(Model):
+        def nsub(self, k, sub):
+            n0 = Model.nsub(self, k, sub)
+            import inspect
+            caller = inspect.stack()[1].function
+            return self.ntiles[k][1] if caller == "softmax" else n0
+
+    assert _caught(Mismatch, units=((1, 2), (3, 4)))
