@@ -5,3 +5,4 @@ this package; the product path never does.
 """
 from .sdpa_ref import default_scale, sdpa, sdpa_packed  # noqa: F401
 from .sdpa_bwd_ref import attention_weights, sdpa_backward, sdpa_backward_packed  # noqa: F401
+from .paged_ref import gather_pages, sdpa_decode_paged  # noqa: F401
