@@ -56,6 +56,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "prefill_tcgen05": ["prefill_sm100.cu", "sm100_ptx.cuh", "exp2_poly.cuh", "common.cuh"],
     "decode_split": ["decode.cu", "common.cuh"],
+    "decode_paged": ["decode.cu", "decode_paged.cu", "common.cuh"],
     "simt": ["simt.cu", "common.cuh"],
     "backward_simt": ["backward_simt.cu", "backward.cuh", "common.cuh"],
     "backward_tcgen05": ["backward_sm100.cu", "backward_simt.cu", "backward.cuh", "tma_host.cuh", "sm100_ptx.cuh",
@@ -390,6 +391,61 @@ def measure_backward(w: W.Workload, steps: int, warmup: int, peaks, peak_src, de
     }
 
 
+PAGE_SIZE = 16
+
+
+def measure_paged_decode(w: W.Workload, steps: int, warmup: int, peaks, peak_src, device):
+    """The decode workload with its key/value cache in pages of 16 tokens of a
+    shared pool, the pages in shuffled order behind each row's block table
+    (sdpa_decode_paged).  Algorithmic bytes: the same K/V bytes as the
+    contiguous decode (the block table adds 4 bytes per page)."""
+    from scaled_dot_product_15_b200 import api, sdpa_decode_paged
+
+    q, k, v = W.make_inputs(w, device)
+    n_pages = w.B * w.S // PAGE_SIZE
+    perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(w.seed)).to(device)
+
+    def pool(t):
+        # (B, Hkv, S, E) -> pages (B*S/16, 16, Hkv, E), page i stored at perm[i]
+        pages = t.transpose(1, 2).reshape(n_pages, PAGE_SIZE, w.Hkv, t.shape[-1])
+        out = torch.empty_like(pages)
+        out[perm] = pages
+        return out
+
+    kp = pool(k)
+    del k
+    vp = pool(v)
+    del v
+    torch.cuda.empty_cache()
+    table = perm.to(torch.int32).reshape(w.B, w.S // PAGE_SIZE).contiguous()
+    lens = torch.full((w.B,), w.S, dtype=torch.int32, device=device)
+    out, lse = sdpa_decode_paged(q, kp, vp, table, lens)
+
+    def call():
+        sdpa_decode_paged(q, kp, vp, table, lens, out=out, lse=lse)
+        return api.last_launch_count()
+
+    total_ms, kernel_ms, launches = time_device([call], steps, warmup, False)
+    amount = W.kv_bytes(w)
+    achieved = rate(amount, kernel_ms, "GB/s")
+    peak = float(peaks["hbm_gbs"])
+    res = {
+        "value": round(rate(amount, total_ms / steps, "GB/s"), 3),
+        "unit": "GB/s",
+        "ms_per_step": round(total_ms / steps, 5),
+        "path": "decode_paged",
+        "gpu_launches": launches,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 3), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": stored_traffic(w.name + f":paged{PAGE_SIZE}", "decode_paged"),
+                     "peak_source": f"of {peak_src}", "algorithmic_per_launch": amount},
+        "note": f"paged cache: pages of {PAGE_SIZE} tokens in shuffled order, one block table per row",
+    }
+    del kp, vp, q, out, lse
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------- CPU oracle
 
 
@@ -526,8 +582,11 @@ def main():
                     help="only run the workload's launches (for profilers); prints no bench line")
     ap.add_argument("--bare-backward", action="store_true",
                     help="time only the workload's backward (gradients) and print one short line (for profilers)")
+    ap.add_argument("--bare-paged", action="store_true",
+                    help="time only the decode workload over a paged cache and print one short line (for profilers)")
     ap.add_argument("--bare-batch", type=int, default=0,
-                    help="with --bare: use this batch size instead of the workload's (smaller profiler captures)")
+                    help="with --bare / --bare-paged: use this batch size instead of the workload's "
+                         "(smaller profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -548,6 +607,15 @@ def main():
     if args.bare_backward:
         r = measure_backward(w, args.steps, args.warmup, peaks, peak_src, device)
         print(json.dumps({"bare_backward": w.name, "ms_per_step": r["ms_per_step"], "path": r["path"],
+                          "launches": r["gpu_launches"]}))
+        return
+    if args.bare_paged:
+        if args.bare_batch:
+            import dataclasses
+
+            w = dataclasses.replace(w, B=args.bare_batch)
+        r = measure_paged_decode(w, args.steps, args.warmup, peaks, peak_src, device)
+        print(json.dumps({"bare_paged": w.name, "ms_per_step": r["ms_per_step"], "path": r["path"],
                           "launches": r["gpu_launches"]}))
         return
     if args.bare:
@@ -585,6 +653,13 @@ def main():
                 extra[w.name + ":backward"] = measure_backward(w, 5, 2, peaks, peak_src, device)
             except Exception as e:
                 extra[w.name + ":backward"] = {"error": repr(e)}
+        for name, ow in W.WORKLOADS.items():
+            if ow.L == 1 and ow.mask == "none" and ow.layout != "packed":
+                try:
+                    extra[name + f":paged{PAGE_SIZE}"] = measure_paged_decode(
+                        ow, max(20, args.steps // 4), args.warmup, peaks, peak_src, device)
+                except Exception as e:
+                    extra[name + f":paged{PAGE_SIZE}"] = {"error": repr(e)}
     if rank == 0 and ws == 1:
         cpu = cpu_baseline(w, args.cpu_seconds)
 

@@ -138,17 +138,19 @@ int sdpa_fwd_plan(int B, int Hq, int Hkv, int L, int S, int E, int Ev,
                   const void* q, const void* k, const void* v, const void* out);
 
 /*
- * Number of kernels the last successful sdpa_fwd() call on this host thread
- * enqueued (1 or 2), for launch accounting in benchmarks.
+ * Number of kernels the last successful sdpa_fwd() or sdpa_decode_paged()
+ * call on this host thread enqueued (1 or 2), for launch accounting in benchmarks.
  */
 int sdpa_last_launch_count(void);
 
 /*
- * Reads and clears the device-side error word of the current device
- * (synchronises the device).  *code receives 0 when no kernel gave up; a
- * non-zero value means a kernel's bounded wait on one of its own pipeline
- * barriers ran out (2 s) and its outputs for that launch are not valid.
- * Returns SDPA_OK, SDPA_ERR_INVALID for a NULL `code`, or SDPA_ERR_CUDA.
+ * Reads and clears the device-side error words of the current device
+ * (synchronises the device).  *code receives 0 when no kernel reported an
+ * error.  Codes below 30 mean a kernel's bounded wait on one of its own
+ * pipeline barriers ran out (2 s) and its outputs for that launch are not
+ * valid; 31 and 32 are sdpa_decode_paged()'s checks of seq_lens and of the
+ * block table.  Returns SDPA_OK, SDPA_ERR_INVALID for a NULL `code`, or
+ * SDPA_ERR_CUDA.
  */
 int sdpa_take_device_error(int* code);
 
@@ -254,6 +256,49 @@ int sdpa_decode_fwd_noalloc(const void* q, const void* k, const void* v, void* o
                             const int64_t q_stride[4], const int64_t k_stride[4],
                             const int64_t v_stride[4], const int64_t o_stride[4],
                             int has_scale, float scale, int dtype, void* stream);
+
+/*
+ * Decode attention over a paged key/value cache.
+ *
+ * Each batch row's keys and values live in fixed-size pages of two shared
+ * pools, found through the row's block table, as in paged KV-cache engines
+ * (the hourtab.com xFormers retainer post, "Related retainer posts", names
+ * them and their failure mode: pages read beyond what a sequence was given,
+ * garbage output, no error).  The keys (values) of row b are the first
+ * seq_lens[b] tokens of pages block_table[b * max_pages + 0],
+ * block_table[b * max_pages + 1], ... taken in table order; the result is the
+ * attention of row b's L query rows over them with no mask, as sdpa_fwd()
+ * computes it (a row with seq_lens[b] = 0 gets O = 0 and lse = -inf).
+ *
+ * Arguments:
+ * - q (B, Hq, L, E), out (B, Hq, L, Ev), lse (B, Hq, L) float32: as for
+ *   sdpa_fwd(), with q_stride / o_stride in (batch, head, row, feature) order.
+ * - k_pages, v_pages: the pools, num_pages pages of page_size tokens and Hkv
+ *   heads each; kp_stride / vp_stride are element strides in the order
+ *   (page, head, token in page, feature), so both (num_pages, page_size,
+ *   Hkv, E) and (num_pages, Hkv, page_size, E) pools are described.
+ * - block_table: device int32 [B][max_pages], row-major; seq_lens: device
+ *   int32 [B].  Both are read on the device, so they may change between
+ *   calls recorded in a CUDA graph.
+ * - page_size: a power of two from 1 to 65536; max_pages * page_size <= 2^20.
+ * - has_scale / scale, dtype, workspace, stream: as for sdpa_fwd(); the
+ *   workspace must hold sdpa_decode_paged_workspace_size() bytes.
+ *
+ * Supported: fp16 / bf16, E = Ev in {64, 128, 256}, (Hq / Hkv) * L <= 8,
+ * 16-byte aligned pointers and strides; SDPA_ERR_UNSUPPORTED otherwise.
+ * Errors found on the device never fault and never read outside the pools:
+ * a table entry outside [0, num_pages) drops that page's tokens and records
+ * code 32, a seq_lens entry outside [0, max_pages * page_size] is clamped
+ * and records code 31; sdpa_take_device_error() returns the code.
+ */
+size_t sdpa_decode_paged_workspace_size(int B, int Hq, int Hkv, int L, int E, int Ev, int page_size,
+                                        int max_pages, int dtype);
+int sdpa_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                      const int32_t* seq_lens, void* out, float* lse, int B, int Hq, int Hkv, int L, int E,
+                      int Ev, int num_pages, int page_size, int max_pages, const int64_t q_stride[4],
+                      const int64_t kp_stride[4], const int64_t vp_stride[4], const int64_t o_stride[4],
+                      int has_scale, float scale, int dtype, void* workspace, size_t workspace_bytes,
+                      void* stream);
 
 #ifdef __cplusplus
 }

@@ -53,8 +53,9 @@ def sdpa_decode_paged(query, k_pages, v_pages, block_table, seq_lens,
     """Attention of query (B, Hq, L, E) over each row's paged keys and
     values.  Returns out (B, Hq, L, Ev) and lse (B, Hq, L)."""
     q = _as_f64(query)
+    k_pages, v_pages = _as_f64(k_pages), _as_f64(v_pages)
     B, Hq, L, E = q.shape
-    Ev = np.asarray(v_pages).shape[-1]
+    Ev = v_pages.shape[-1]
     out = np.empty((B, Hq, L, Ev))
     lse = np.empty((B, Hq, L))
     for b in range(B):

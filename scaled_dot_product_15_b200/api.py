@@ -73,6 +73,12 @@ _SIGNATURES = {
         [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 + [_I64x4] * 4
         + [ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p],
     ),
+    "sdpa_decode_paged_workspace_size": (ctypes.c_size_t, [ctypes.c_int] * 9),
+    "sdpa_decode_paged": (
+        ctypes.c_int,
+        [ctypes.c_void_p] * 7 + [ctypes.c_int] * 9 + [_I64x4] * 4
+        + [ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
+    ),
 }
 
 _lib = None
@@ -433,8 +439,88 @@ def plan(query, key, value, *, layout="bhle", mask_kind=MASK_NONE, out=None) -> 
     return PLAN_NAMES[r]
 
 
+def sdpa_decode_paged(
+    query: torch.Tensor,
+    k_pages: torch.Tensor,
+    v_pages: torch.Tensor,
+    block_table: torch.Tensor,
+    seq_lens: torch.Tensor,
+    scale: Optional[float] = None,
+    *,
+    pages_layout: str = "token_major",
+    out: Optional[torch.Tensor] = None,
+    lse: Optional[torch.Tensor] = None,
+) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Decode attention of query (B, Hq, L, E) over a paged key/value cache.
+
+    Row b's keys and values are the first ``seq_lens[b]`` tokens of pages
+    ``block_table[b, 0], block_table[b, 1], ...`` of the pools (see
+    sdpa_decode_paged in include/sdpa15.h).  ``pages_layout="token_major"``:
+    pools (num_pages, page_size, Hkv, E); ``"head_major"``: (num_pages, Hkv,
+    page_size, E).  block_table (B, max_pages) and seq_lens (B,) are int32 on
+    the device.  Returns ``(out, lse)``: out (B, Hq, L, Ev), lse float32
+    (B, Hq, L).  Query heads are grouped over key/value heads (Hq a multiple
+    of Hkv).
+    """
+    lib = load_library()
+    if query.dim() != 4 or k_pages.dim() != 4 or v_pages.dim() != 4:
+        raise ValueError("query and the page pools must be 4-D")
+    if not (query.dtype == k_pages.dtype == v_pages.dtype) or query.dtype not in _DTYPE_CODE:
+        raise ValueError("query and the page pools must share a supported dtype")
+    for t, name in ((block_table, "block_table"), (seq_lens, "seq_lens")):
+        if t.dtype != torch.int32 or not t.is_cuda:
+            raise ValueError(f"{name} must be an int32 CUDA tensor")
+    if not (query.is_cuda and k_pages.is_cuda and v_pages.is_cuda):
+        raise ValueError("inputs must be CUDA tensors")
+    B, Hq, L, E = query.shape
+    if pages_layout == "token_major":
+        num_pages, page_size, Hkv, Ek = k_pages.shape
+        perm = (0, 2, 1, 3)
+    elif pages_layout == "head_major":
+        num_pages, Hkv, page_size, Ek = k_pages.shape
+        perm = (0, 1, 2, 3)
+    else:
+        raise ValueError(f"unknown pages_layout {pages_layout!r}")
+    Ev = v_pages.shape[-1]
+    if Ek != E or tuple(v_pages.shape[:3]) != tuple(k_pages.shape[:3]):
+        raise ValueError("query and page pool shapes do not agree")
+    if Hkv == 0 or Hq % Hkv != 0:
+        raise ValueError("query heads must be a multiple of key/value heads")
+    if block_table.dim() != 2 or block_table.shape[0] != B or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous (B, max_pages) tensor")
+    if seq_lens.shape != (B,) or not seq_lens.is_contiguous():
+        raise ValueError("seq_lens must be a contiguous (B,) tensor")
+    max_pages = block_table.shape[1]
+    dev = query.device
+    dcode = _DTYPE_CODE[query.dtype]
+    if out is None:
+        out = torch.empty((B, Hq, L, Ev), dtype=query.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    if not lse.is_contiguous() or lse.dtype != torch.float32:
+        raise ValueError("lse must be a contiguous float32 tensor")
+    ks_, vs_ = (tuple(t.stride(d) for d in perm) for t in (k_pages, v_pages))
+    qs, os_ = _i64x4(query.stride()), _i64x4(out.stride())
+    ws_bytes = lib.sdpa_decode_paged_workspace_size(B, Hq, Hkv, L, E, Ev, page_size, max_pages, dcode)
+    ws = _workspace(dev, ws_bytes)
+    ws_ptr = None if ws is None else (ws.data_ptr() + 255) // 256 * 256
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        status = lib.sdpa_decode_paged(
+            query.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
+            seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(),
+            B, Hq, Hkv, L, E, Ev, num_pages, page_size, max_pages,
+            qs, _i64x4(ks_), _i64x4(vs_), os_,
+            0 if scale is None else 1, 0.0 if scale is None else float(scale),
+            dcode, ws_ptr, ws_bytes, stream,
+        )
+    _check(status, "sdpa_decode_paged")
+    return out, lse
+
+
 def take_device_error() -> int:
-    """Device-side error word (0 = no kernel gave up on a wait), cleared."""
+    """Device-side error word (0 = none; below 30: a kernel gave up on a
+    wait; 31 / 32: a paged decode's seq_lens / block table check), cleared."""
     code = ctypes.c_int(0)
     _check(load_library().sdpa_take_device_error(ctypes.byref(code)), "sdpa_take_device_error")
     return code.value

@@ -18,9 +18,33 @@
 // chunk a second kernel merges them:  lse = log2 sum_s 2^lse_s  and
 // O = sum_s 2^(lse_s - lse) O_s  (the logsumexp-merge identity: each chunk's
 // softmax restricted to its keys, reweighted by its share of the total).
+//
+// Paged caches: the same kernels read a row's keys and values from pages of a
+// shared pool through its block table (kPaged).  Row b's keys are the first
+// seq_lens[b] tokens of pages block_table[b][0], block_table[b][1], ... in
+// table order; the hourtab.com xFormers retainer post ("Related retainer
+// posts") recalls engines reading pages past a sequence's allocation and
+// returning garbage with no error, so here every table entry is checked
+// against the pool before use: an entry outside it drops that page's tokens
+// and records error 32 in the decode error word, a length outside
+// [0, max_pages * page_size] is clamped and records error 31.  No address
+// outside the pool is ever formed.
 #include "common.cuh"
 
 namespace sdpa15 {
+
+// Error word of the decode kernels (0 = none), read and cleared by
+// decode_take_error().
+__device__ int g_decode_error = 0;
+
+// Block table of a paged cache (all zero for a contiguous one).
+struct PagedArgs {
+  const int32_t* table;  // [B][max_pages] page indices into the pool
+  const int32_t* lens;   // [B] tokens per row
+  int max_pages;
+  int num_pages;         // pages in the pool
+  int shift;             // log2(page_size)
+};
 
 constexpr int kDecThreads = 256;
 constexpr int kDecChunkMax = 1024;  // keys per CTA at most
@@ -101,9 +125,9 @@ __device__ __forceinline__ float group_reduce_rows(float (&v)[R], int lane, int&
   return v[0];
 }
 
-template <typename T, int E, int R>
+template <typename T, int E, int R, bool kPaged>
 __global__ void __launch_bounds__(kDecThreads, (R <= 4 ? 3 : 2))
-decode_split_kernel(Params p, int nsplit, int chunk) {
+decode_split_kernel(Params p, int nsplit, int chunk, PagedArgs pg) {
   constexpr int G = E / 8;              // lanes per key row (16-byte slices)
   constexpr int KPW = 32 / G;           // keys per warp step
   constexpr int NKG = kDecThreads / G;  // lane groups per CTA
@@ -112,15 +136,55 @@ decode_split_kernel(Params p, int nsplit, int chunk) {
   float* lg = smem;  // [chunk][R] base-2 logits, then weights; reused for the reduction
   __shared__ float s_max[R], s_sum[R];
   __shared__ int s_flag[R];  // 1: NaN logit, 2: +inf logit
+  // Paged: the pool index of each page this chunk touches (-1: an entry
+  // outside the pool).
+  __shared__ int s_page[kPaged ? kDecChunkMax + 2 : 1];
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int s0 = split * chunk;
-  const int s1 = min(p.S, s0 + chunk);
-  const int n = max(0, s1 - s0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int S_b = p.S;
+  if constexpr (kPaged) {
+    const int len = __ldg(pg.lens + b);
+    S_b = min(max(len, 0), p.S);  // p.S = max_pages * page_size
+    if (S_b != len && tid == 0 && split == 0 && kvh == 0) atomicCAS(&g_decode_error, 0, 31);
+  }
+  const int s0 = split * chunk;
+  const int s1 = min(S_b, s0 + chunk);
+  const int n = max(0, s1 - s0);
+  const int first_page = kPaged ? (s0 >> pg.shift) : 0;
+  if constexpr (kPaged) {
+    // The host keeps rows within 2^20 tokens, so a chunk holds at most 1024
+    // keys and touches at most kDecChunkMax + 2 pages.
+    const int count = n > 0 ? min(((s0 + n - 1) >> pg.shift) - first_page + 1, kDecChunkMax + 2) : 0;
+    for (int i = tid; i < count; i += kDecThreads) {
+      const int e = __ldg(pg.table + (int64_t)b * pg.max_pages + first_page + i);
+      const bool ok = e >= 0 && e < pg.num_pages;
+      if (!ok) atomicCAS(&g_decode_error, 0, 32);
+      s_page[i] = ok ? e : -1;
+    }
+    __syncthreads();
+  }
+  // Element offset of key/value token j of this chunk from chunk_base(), or
+  // -1 when its page is not in the pool.
+  auto token_offset = [&](int j, const int64_t* st) -> int64_t {
+    if constexpr (kPaged) {
+      const int tok = s0 + j;
+      const int page = s_page[(tok >> pg.shift) - first_page];
+      if (page < 0) return -1;
+      return (int64_t)page * st[0] + (int64_t)(tok & ((1 << pg.shift) - 1)) * st[2];
+    } else {
+      return (int64_t)(s0 + j) * st[2];
+    }
+  };
   const int gl = lane % G;                 // lane within its group
   const int kg = warp * KPW + lane / G;    // group index
   const int rows = p.group * p.L;          // live rows (<= R)
+  // Contiguous cache: this batch row's keys; paged: the pool.
+  auto chunk_base = [&](const void* base, const int64_t* st) -> const T* {
+    const T* b0 = static_cast<const T*>(base) + kvh * st[1] + gl * 8;
+    if constexpr (kPaged) return b0;
+    else return b0 + b * st[0];
+  };
 
   // Query rows: row r = (query head kvh*group + r / L, position r % L).
   float qf[R][8];
@@ -139,7 +203,7 @@ decode_split_kernel(Params p, int nsplit, int chunk) {
   }
 
   // Phase 1: logits.
-  const T* kbase = static_cast<const T*>(p.k) + b * p.ks[0] + kvh * p.ks[1] + gl * 8;
+  const T* kbase = chunk_base(p.k, p.ks);
   // The loop bound is warp-uniform (the shuffles below need every lane).
   for (int jb = warp * KPW; jb < n; jb += NKG * kDecUnroll) {
     const int j0 = jb + lane / G;
@@ -147,7 +211,8 @@ decode_split_kernel(Params p, int nsplit, int chunk) {
 #pragma unroll
     for (int u = 0; u < kDecUnroll; ++u) {
       const int j = j0 + u * NKG;
-      if (j < n) raw[u] = Vec8<T>::raw(kbase + (int64_t)(s0 + j) * p.ks[2]);
+      const int64_t off = j < n ? token_offset(j, p.ks) : -1;
+      if (off >= 0) raw[u] = Vec8<T>::raw(kbase + off);
       else raw[u] = make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
@@ -166,7 +231,11 @@ decode_split_kernel(Params p, int nsplit, int chunk) {
       int row;
       const float full = group_reduce_rows<R, G>(d, gl, row);
       // lanes holding a replica of the same row: the first one writes
-      if (j < n && (gl % (G / R > 0 ? G / R : 1)) == 0) lg[j * R + row] = full;
+      if (j < n && (gl % (G / R > 0 ? G / R : 1)) == 0) {
+        bool dropped = false;  // paged: the key's page is not in the pool
+        if constexpr (kPaged) dropped = s_page[((s0 + j) >> pg.shift) - first_page] < 0;
+        lg[j * R + row] = dropped ? -INFINITY : full;
+      }
     }
   }
   __syncthreads();
@@ -201,14 +270,15 @@ decode_split_kernel(Params p, int nsplit, int chunk) {
   for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
-  const T* vbase = static_cast<const T*>(p.v) + b * p.vs[0] + kvh * p.vs[1] + gl * 8;
+  const T* vbase = chunk_base(p.v, p.vs);
   for (int jb = warp * KPW; jb < n; jb += NKG * kDecUnroll) {
     const int j0 = jb + lane / G;
     uint4 raw[kDecUnroll];
 #pragma unroll
     for (int u = 0; u < kDecUnroll; ++u) {
       const int j = j0 + u * NKG;
-      if (j < n) raw[u] = Vec8<T>::raw(vbase + (int64_t)(s0 + j) * p.vs[2]);
+      const int64_t off = j < n ? token_offset(j, p.vs) : -1;
+      if (off >= 0) raw[u] = Vec8<T>::raw(vbase + off);
       else raw[u] = make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
@@ -329,8 +399,8 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int L, int S, int Ev) {
   return (size_t)ns * nrows * ((size_t)Ev + 1) * sizeof(float);
 }
 
-template <typename T, int E, int R>
-static cudaError_t launch_decode_t(const Params& p, cudaStream_t st, int* launches) {
+template <typename T, int E, int R, bool kPaged>
+static cudaError_t launch_decode_t(const Params& p, const PagedArgs& pg, cudaStream_t st, int* launches) {
   const int ns = decode_splits(p.B, p.Hkv, p.S);
   const int chunk = (p.S + ns - 1) / ns;
   constexpr int G = E / 8;
@@ -338,11 +408,11 @@ static cudaError_t launch_decode_t(const Params& p, cudaStream_t st, int* launch
   const size_t smem_lg = (size_t)chunk * R * sizeof(float);
   const size_t smem_red = (size_t)NKG * R * E * sizeof(float);
   const size_t smem = smem_lg > smem_red ? smem_lg : smem_red;
-  auto kern = decode_split_kernel<T, E, R>;
+  auto kern = decode_split_kernel<T, E, R, kPaged>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid(ns, p.Hkv, p.B);
-  kern<<<grid, kDecThreads, smem, st>>>(p, ns, chunk);
+  kern<<<grid, kDecThreads, smem, st>>>(p, ns, chunk, pg);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   *launches = 1;
@@ -355,21 +425,21 @@ static cudaError_t launch_decode_t(const Params& p, cudaStream_t st, int* launch
   return err;
 }
 
-template <typename T, int E>
-static cudaError_t launch_decode_e(const Params& p, cudaStream_t st, int* launches) {
+template <typename T, int E, bool kPaged>
+static cudaError_t launch_decode_e(const Params& p, const PagedArgs& pg, cudaStream_t st, int* launches) {
   const int rows = p.group * p.L;
-  if (rows <= 1) return launch_decode_t<T, E, 1>(p, st, launches);
-  if (rows <= 2) return launch_decode_t<T, E, 2>(p, st, launches);
-  if (rows <= 4) return launch_decode_t<T, E, 4>(p, st, launches);
-  return launch_decode_t<T, E, 8>(p, st, launches);
+  if (rows <= 1) return launch_decode_t<T, E, 1, kPaged>(p, pg, st, launches);
+  if (rows <= 2) return launch_decode_t<T, E, 2, kPaged>(p, pg, st, launches);
+  if (rows <= 4) return launch_decode_t<T, E, 4, kPaged>(p, pg, st, launches);
+  return launch_decode_t<T, E, 8, kPaged>(p, pg, st, launches);
 }
 
-template <typename T>
-static cudaError_t launch_decode_d(const Params& p, cudaStream_t st, int* launches) {
+template <typename T, bool kPaged>
+static cudaError_t launch_decode_d(const Params& p, const PagedArgs& pg, cudaStream_t st, int* launches) {
   switch (p.E) {
-    case 64: return launch_decode_e<T, 64>(p, st, launches);
-    case 128: return launch_decode_e<T, 128>(p, st, launches);
-    default: return launch_decode_e<T, 256>(p, st, launches);
+    case 64: return launch_decode_e<T, 64, kPaged>(p, pg, st, launches);
+    case 128: return launch_decode_e<T, 128, kPaged>(p, pg, st, launches);
+    default: return launch_decode_e<T, 256, kPaged>(p, pg, st, launches);
   }
 }
 
@@ -392,8 +462,26 @@ bool decode_supported(const Params& p, int dtype) {
 }
 
 cudaError_t launch_decode(const Params& p, int dtype, cudaStream_t st, int* launches) {
-  if (dtype == SDPA_F16) return launch_decode_d<__half>(p, st, launches);
-  return launch_decode_d<__nv_bfloat16>(p, st, launches);
+  const PagedArgs none = {nullptr, nullptr, 0, 0, 0};
+  if (dtype == SDPA_F16) return launch_decode_d<__half, false>(p, none, st, launches);
+  return launch_decode_d<__nv_bfloat16, false>(p, none, st, launches);
+}
+
+// Paged cache: p.k / p.v are the page pools with strides (page, head, token
+// in page, feature), p.S = max_pages * page_size; decode_supported(p) holds.
+cudaError_t launch_decode_paged(const Params& p, const int32_t* table, const int32_t* lens, int max_pages,
+                                int num_pages, int page_shift, int dtype, cudaStream_t st, int* launches) {
+  const PagedArgs pg = {table, lens, max_pages, num_pages, page_shift};
+  if (dtype == SDPA_F16) return launch_decode_d<__half, true>(p, pg, st, launches);
+  return launch_decode_d<__nv_bfloat16, true>(p, pg, st, launches);
+}
+
+// Reads and clears the decode kernels' error word.  Synchronous.
+cudaError_t decode_take_error(int* code) {
+  int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_decode_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_decode_error, &zero, sizeof(int));
 }
 
 }  // namespace sdpa15

@@ -20,6 +20,7 @@ cudaError_t launch_rowdot(const Params& p, const BwdParams& g, int dtype, cudaSt
 bool backward_sm100_supported(const Params& p, const BwdParams& g, int dtype);
 cudaError_t launch_backward_sm100(const Params& p, const BwdParams& g, int dtype, cudaStream_t st);
 cudaError_t backward_take_error(int* code);
+cudaError_t decode_take_error(int* code);
 }  // namespace sdpa15
 
 using namespace sdpa15;
@@ -85,6 +86,11 @@ bool is_sm100() {
 
 }  // namespace
 
+namespace sdpa15 {
+// Kernel launches of this thread's last call (for sdpa_last_launch_count).
+void set_last_launches(int n) { t_last_launches = n; }
+}  // namespace sdpa15
+
 extern "C" {
 
 int sdpa_abi_version(void) { return kAbiVersion; }
@@ -106,9 +112,11 @@ int sdpa_take_device_error(int* code) {
   if (!code) return SDPA_ERR_INVALID;
   *code = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return SDPA_ERR_CUDA;
-  int c1 = 0, c2 = 0;
-  if (prefill_take_error(&c1) != cudaSuccess || backward_take_error(&c2) != cudaSuccess) return SDPA_ERR_CUDA;
-  *code = c1 ? c1 : c2;
+  int c1 = 0, c2 = 0, c3 = 0;
+  if (prefill_take_error(&c1) != cudaSuccess || backward_take_error(&c2) != cudaSuccess ||
+      decode_take_error(&c3) != cudaSuccess)
+    return SDPA_ERR_CUDA;
+  *code = c1 ? c1 : (c2 ? c2 : c3);
   return SDPA_OK;
 }
 

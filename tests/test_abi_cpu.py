@@ -145,3 +145,44 @@ def test_backward_host_side_rejections_and_workspace():
         assert _bwd(ws=0x10100, ws_bytes=256) == api.SDPA_ERR_UNSUPPORTED
     assert _bwd(ws=0x10180, ws_bytes=256) == api.SDPA_ERR_WORKSPACE  # not 256-byte aligned
     assert _bwd(B=0) == api.SDPA_OK
+
+
+def _paged(B=2, Hq=8, Hkv=2, L=1, E=128, Ev=128, num_pages=16, page_size=16, max_pages=4, dtype=api.SDPA_BF16,
+           kstride=None, scale=None, ptr=0x100000, table=0x200000):
+    lib = api.load_library()
+    qs = api._i64x4((Hq * L * E, L * E, E, 1))
+    ks = api._i64x4(kstride or (page_size * Hkv * E, E, Hkv * E, 1))  # token-major pool
+    os_ = api._i64x4((Hq * L * Ev, L * Ev, Ev, 1))
+    return lib.sdpa_decode_paged(ptr, ptr, ptr, table, table, ptr, ptr, B, Hq, Hkv, L, E, Ev, num_pages, page_size,
+                                 max_pages, qs, ks, ks, os_, 0 if scale is None else 1, scale or 0.0, dtype,
+                                 None, 0, None)
+
+
+def test_paged_decode_host_side_rejections_and_workspace():
+    assert _paged(Hq=3, Hkv=2) == api.SDPA_ERR_INVALID           # Hq not a multiple of Hkv
+    assert _paged(page_size=24) == api.SDPA_ERR_UNSUPPORTED      # not a power of two
+    assert _paged(page_size=0) == api.SDPA_ERR_INVALID
+    assert _paged(max_pages=0) == api.SDPA_ERR_INVALID
+    assert _paged(num_pages=0) == api.SDPA_ERR_INVALID
+    assert _paged(dtype=api.SDPA_F32) == api.SDPA_ERR_UNSUPPORTED  # 16-bit only
+    assert _paged(E=96, Ev=96) == api.SDPA_ERR_UNSUPPORTED       # E in {64, 128, 256}
+    assert _paged(Hq=16, Hkv=1) == api.SDPA_ERR_UNSUPPORTED      # more than 8 rows per key/value head
+    assert _paged(kstride=(1, 1, 1, 2)) == api.SDPA_ERR_INVALID  # feature stride must be 1
+    assert _paged(kstride=(16, 8, 4, 1)) == api.SDPA_ERR_UNSUPPORTED  # rows not 16-byte aligned
+    assert _paged(scale=float("inf")) == api.SDPA_ERR_INVALID
+    assert _paged(ptr=None) == api.SDPA_ERR_INVALID
+    assert _paged(table=None) == api.SDPA_ERR_INVALID
+    assert _paged(B=0, ptr=None, table=None) == api.SDPA_OK       # empty problem
+    lib = api.load_library()
+    n = lib.sdpa_decode_paged_workspace_size(64, 32, 8, 1, 128, 128, 16, 1024, api.SDPA_BF16)
+    assert n > 0 and n == lib.sdpa_fwd_workspace_size(64, 32, 8, 1, 16384, 128, 128, api.MASK_NONE, api.SDPA_BF16)
+    assert lib.sdpa_decode_paged_workspace_size(64, 32, 8, 1, 128, 128, 24, 1024, api.SDPA_BF16) == 0
+    assert _paged(B=64, Hq=32, Hkv=8, max_pages=1024, num_pages=65536) == api.SDPA_ERR_WORKSPACE  # needs scratch
+
+
+def test_paged_decode_without_gpu_is_unsupported():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _paged() == api.SDPA_ERR_UNSUPPORTED
