@@ -44,8 +44,10 @@
 //               are already being computed.
 // Causal attention visits only key tiles at or left of the diagonal, per
 // sub-tile: the last key tile of a 256-row unit lies wholly above sub-tile 0's
-// rows, so sub-tile 0 skips its scores, softmax and PV.  Packed
-// variable-length batches index tiles from each segment's first token.
+// rows, so sub-tile 0 skips its scores, softmax and PV.  A unit whose
+// sub-tile 1 has no rows (the last block of a short segment or sequence)
+// skips all of sub-tile 1's work.  Packed variable-length batches index tiles
+// from each segment's first token.
 //
 // Every wait on an mbarrier is bounded (2 s); on a timeout the kernel records
 // an error code, stops its other roles, drains what it issued and returns.
@@ -131,9 +133,10 @@ static_assert(sizeof(Bars) <= 512, "barrier block");
 // A work unit: 256 query rows of one (batch or segment, head).
 struct Unit {
   int h, b, seq0, Lq, Sk, row0;
-  int n_kv;  // key tiles of the unit (sub-tile 1's)
+  int n_kv;  // key tiles of the unit
   int n0;    // key tiles of sub-tile 0: n_kv, or n_kv - 1 under a causal mask
              // when the last tile lies wholly above sub-tile 0's rows
+  int n1;    // key tiles of sub-tile 1: n_kv, or 0 when it has no rows
 };
 
 template <typename T>
@@ -350,6 +353,7 @@ __device__ __forceinline__ bool unit_at(const Params& p, int idx, int bx, int mb
   }
   u.n_kv = n;
   u.n0 = n0;
+  u.n1 = u.row0 + BM < u.Lq ? n : 0;
   return true;
 }
 
@@ -552,14 +556,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ok = mma_wait<kWI>(bars, &bars->full[0], 0);
 #pragma unroll 1
         for (int sub = 0; sub < NSUB && ok; ++sub) {
+          // A sub-tile without tiles still takes its Q barrier's phase.
           if (!mma_wait<kWI>(bars, &bars->q[sub], 0)) {
             ok = false;
             break;
           }
-          ptx::tc_fence_after();
-          issue_qk<D, kWI>(tmem + sub * 128, dq + sub * kSubStep, dk0, idesc_qk);
-          mma_commit_as<kWI>(&bars->s[sub]);
-          if ((sub ? u.n_kv : u.n0) == 1) mma_commit_as<kWI>(&bars->q_free[sub]);
+          const int ns = sub ? u.n1 : u.n0;
+          if (ns > 0) {
+            ptx::tc_fence_after();
+            issue_qk<D, kWI>(tmem + sub * 128, dq + sub * kSubStep, dk0, idesc_qk);
+            mma_commit_as<kWI>(&bars->s[sub]);
+          }
+          if (ns <= 1) mma_commit_as<kWI>(&bars->q_free[sub]);
         }
         if (ok) mma_commit_as<kWI>(&bars->empty[0]);
       }
@@ -589,16 +597,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             mma_commit_as<kWI>(&bars->s[0]);
             if (j + 2 == u.n0) mma_commit_as<kWI>(&bars->q_free[0]);  // its last scores of the unit
           }
-          if (!mma_wait<kWI>(bars, &bars->p[1], tile1 & 1)) {
-            ok = false;
-            break;
+          if (u.n1 > 0) {  // sub-tile 1 may have no rows (a short segment's last block)
+            if (!mma_wait<kWI>(bars, &bars->p[1], tile1 & 1)) {
+              ok = false;
+              break;
+            }
+            ++tile1;
+            ptx::tc_fence_after();
+            issue_pv<kWI>(tmem + 384, tmem + 128, dv, acc, idesc_pv);
+            issue_qk<D, kWI>(tmem + 128, dq + kSubStep, dk, idesc_qk);
+            mma_commit_as<kWI>(&bars->s[1]);
+            if (j + 2 == n) mma_commit_as<kWI>(&bars->q_free[1]);
           }
-          ++tile1;
-          ptx::tc_fence_after();
-          issue_pv<kWI>(tmem + 384, tmem + 128, dv, acc, idesc_pv);
-          issue_qk<D, kWI>(tmem + 128, dq + kSubStep, dk, idesc_qk);
-          mma_commit_as<kWI>(&bars->s[1]);
-          if (j + 2 == n) mma_commit_as<kWI>(&bars->q_free[1]);
           mma_commit_as<kWI>(&bars->empty[vslot]);
           mma_commit_as<kWI>(&bars->empty[kslot]);
         }
@@ -616,7 +626,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (nx_have) unit_at<kVarlen>(p, nidx, bx, mblocks, causal, nx);
 #pragma unroll 1
         for (int sub = 0; sub < NSUB; ++sub) {
-          if (sub == 1 || u.n0 == n) {
+          if ((sub ? u.n1 : u.n0) == n) {
             if (!mma_wait<kWI>(bars, &bars->p[sub], (sub ? tile1 : tile0) & 1)) {
               ok = false;
               break;
@@ -634,10 +644,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             ok = false;
             break;
           }
-          ptx::tc_fence_after();
-          issue_qk<D, kWI>(tmem + sub * 128, dq + sub * kSubStep, dk0 + kslot * kSlotStep, idesc_qk);
-          mma_commit_as<kWI>(&bars->s[sub]);
-          if ((sub ? nx.n_kv : nx.n0) == 1) mma_commit_as<kWI>(&bars->q_free[sub]);  // the next unit's last scores
+          const int ns = sub ? nx.n1 : nx.n0;
+          if (ns > 0) {
+            ptx::tc_fence_after();
+            issue_qk<D, kWI>(tmem + sub * 128, dq + sub * kSubStep, dk0 + kslot * kSlotStep, idesc_qk);
+            mma_commit_as<kWI>(&bars->s[sub]);
+          }
+          if (ns <= 1) mma_commit_as<kWI>(&bars->q_free[sub]);  // the next unit's last scores
         }
         if (!ok) break;
         mma_commit_as<kWI>(&bars->empty[vslot]);
@@ -675,7 +688,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int row_lo = u.row0 + sub * BM;
       const int r = row_lo + rin;  // query row within the sequence
       float m_run = -INFINITY, l_run = 0.f;
-      const int n_sub = sub ? u.n_kv : u.n0;
+      const int n_sub = sub ? u.n1 : u.n0;
       for (int j = 0; j < n_sub; ++j, ++tile) {
         // Every wait's outcome is made warp-uniform, so a timeout can never
         // leave part of a warp inside a warp-collective tcgen05 instruction.

@@ -18,10 +18,12 @@ against a model of the hardware:
   once every earlier MMA has executed;
 * TMA loads land at arbitrary later times.
 
-A unit is given as its number of key tiles n, or as (n0, n) when sub-tile 0
-needs only its first n0 = n - 1 tiles (under a causal mask the last key tile
-of a 256-row block lies wholly above sub-tile 0's rows, and the kernel skips
-that tile's scores, softmax and PV for it).
+A unit is given as its number of key tiles n, or as (n0, n1), the tiles each
+sub-tile takes: n0 = n - 1 when under a causal mask the last key tile of a
+256-row block lies wholly above sub-tile 0's rows, n1 = 0 when a short
+segment leaves sub-tile 1 without rows; the kernel skips those tiles' scores,
+softmax and PV (a sub-tile without tiles still takes its Q load and its
+output barrier, so every barrier keeps one phase per unit).
 
 Random interleavings are explored for several unit lists.  Besides deadlock and
 aliasing, every buffer (Q_i, the key/value ring slots, S/P and O in tensor
@@ -71,7 +73,7 @@ class Model:
 
     def __init__(self, units, ns, rng):
         self.ntiles = [u if isinstance(u, tuple) else (u, u) for u in units]
-        self.units = [u[1] for u in self.ntiles]
+        self.units = [max(u) for u in self.ntiles]
         self.ns, self.rng = ns, rng
         B = Bar
         self.q = [B(f"q{a}", 1) for a in range(2)]
@@ -88,7 +90,8 @@ class Model:
         self.qbuf = [None, None]         # tag of each Q_sub buffer
         self.sbuf = [None, None]         # tag in each S/P tensor-memory buffer
         self.obuf = [None, None]         # (unit, PVs applied) in each O buffer
-        self.o_read = [None, None]       # last unit whose O was read out
+        self.o_read = [None, None]       # last unit whose output step ran
+        self.o_consumed = [None, None]   # unit of the O buffer contents last read out
         self.s_exec = [(-1, 0), (-1, 0)]  # last (unit, tile) S MMA executed per sub-tile
         self.pipe = []                   # in-order tensor pipe
         self.tma = []                    # (slot, tag) loads in flight
@@ -133,7 +136,7 @@ class Model:
             if self.sbuf[sub] != ("P", k, j):
                 raise ProtocolError(f"PV{sub}({k},{j}) reads a buffer holding {self.sbuf[sub]}")
             if j == 0:
-                if self.obuf[sub] is not None and self.o_read[sub] != self.obuf[sub][0]:
+                if self.obuf[sub] is not None and self.o_consumed[sub] != self.obuf[sub][0]:
                     raise ProtocolError(f"PV{sub}({k},0) overwrites O of unit {self.obuf[sub][0]} before it was read out")
                 self.obuf[sub] = (k, 1)
             else:
@@ -178,7 +181,7 @@ class Model:
                         for sub in range(2):
                             if nq[sub] > 0:
                                 yield ("wait", self.q_free[sub], (nq[sub] - 1) & 1, nq[sub] - 1)
-                                if self.s_exec[sub] < (k - 1, self.nsub(k - 1, sub) - 1):
+                                if self.nsub(k - 1, sub) > 0 and self.s_exec[sub] < (k - 1, self.nsub(k - 1, sub) - 1):
                                     raise ProtocolError(f"Q{sub} of unit {k} loaded under pending score MMAs of unit {k - 1}")
                             self.qbuf[sub] = ("loading",)
                             self.tma.append((f"q{sub}", ("Q", k)))
@@ -208,9 +211,10 @@ class Model:
         yield ("wait", self.full[0], 0, 0)
         for sub in range(2):
             yield ("wait", self.q[sub], 0, 0)
-            self.pipe.append(("qk", sub, 0, cur, 0))
-            self.pipe.append(("commit", self.s[sub]))
-            if self.nsub(cur, sub) == 1:
+            if self.nsub(cur, sub) > 0:
+                self.pipe.append(("qk", sub, 0, cur, 0))
+                self.pipe.append(("commit", self.s[sub]))
+            if self.nsub(cur, sub) <= 1:
                 self.pipe.append(("commit", self.q_free[sub]))
         self.pipe.append(("commit", self.empty[0]))
         while True:
@@ -222,6 +226,8 @@ class Model:
                 yield ("wait", self.full[vslot], (vt // ns) & 1, vt // ns)
                 for sub in range(2):
                     nsub = self.nsub(cur, sub)
+                    if nsub == 0:
+                        continue
                     yield ("wait", self.p[sub], tile[sub] & 1, tile[sub])
                     tile[sub] += 1
                     self.pipe.append(("pv", sub, vslot, cur, j))
@@ -250,9 +256,10 @@ class Model:
                 if sub == 0:
                     yield ("wait", self.full[kslot], (kt // ns) & 1, kt // ns)
                 yield ("wait", self.q[sub], (k + 1) & 1, k + 1)
-                self.pipe.append(("qk", sub, kslot, nxt, 0))
-                self.pipe.append(("commit", self.s[sub]))
-                if self.nsub(nxt, sub) == 1:
+                if self.nsub(nxt, sub) > 0:
+                    self.pipe.append(("qk", sub, kslot, nxt, 0))
+                    self.pipe.append(("commit", self.s[sub]))
+                if self.nsub(nxt, sub) <= 1:
                     self.pipe.append(("commit", self.q_free[sub]))
             self.pipe.append(("commit", self.empty[vslot]))
             if nxt < 0:
@@ -280,9 +287,11 @@ class Model:
                 tile += 1
             # the unit's output of this sub-tile
             yield ("wait", self.o[sub], k & 1, k)
-            if self.obuf[sub] != (cur, n):
+            if n > 0 and self.obuf[sub] != (cur, n):
                 raise ProtocolError(f"output({cur},{sub}) reads O holding {self.obuf[sub]}")
             self.o_read[sub] = cur
+            if self.obuf[sub] is not None:
+                self.o_consumed[sub] = self.obuf[sub][0]
             k += 1
 
     def run(self):
@@ -322,7 +331,9 @@ class Model:
 UNIT_LISTS = [[1], [2], [3], [5], [16], [33], [1, 1, 1], [3, 1, 2], [5, 5], [1, 4, 2, 6, 1], [16, 8, 2], [2, 2, 2, 2, 2],
               # sub-tile 0 skipping the last key tile (causal row blocks)
               [(1, 2)], [(15, 16), (7, 8), (1, 2)], [(1, 2), (1, 2), (1, 2)], [(3, 4), 2, (1, 2), 1, (5, 6)],
-              [1, (1, 2), (2, 3), 3]]
+              [1, (1, 2), (2, 3), 3],
+              # sub-tile 1 without rows (short last row block of a segment)
+              [(1, 0)], [(3, 0), 2, (2, 0), (1, 2), (4, 0)], [(5, 0), (5, 0)], [(1, 0), (1, 0), (1, 2), (2, 0)]]
 
 
 @pytest.mark.parametrize("units", UNIT_LISTS, ids=lambda u: "-".join(map(str, u)).replace(" ", ""))
@@ -426,3 +437,17 @@ def test_model_catches_a_skipped_tile_still_waited_for():
             return self.ntiles[k][1] if caller == "softmax" else n0
 
     assert _caught(Mismatch, units=((1, 2), (3, 4)))
+
+
+def test_model_catches_a_skipped_q_wait_for_an_empty_sub_tile():
+    """Not waiting for Q_1 of a unit whose sub-tile 1 has no rows lets the
+    next unit's wait on the same barrier pass on the wrong phase."""
+
+    class SkipWait(Model):
+        def mma(self):
+            for item in Model.mma(self):
+                if item[1] is self.q[1] and self.nsub(item[3], 1) == 0:
+                    continue
+                yield item
+
+    assert _caught(SkipWait, units=((2, 0), (1, 2), (3, 0), (2, 3)))
