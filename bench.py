@@ -394,10 +394,13 @@ def measure_backward(w: W.Workload, steps: int, warmup: int, peaks, peak_src, de
 PAGE_SIZE = 16
 
 
-def measure_paged_decode(w: W.Workload, steps: int, warmup: int, peaks, peak_src, device):
+def measure_paged_decode(w: W.Workload, steps: int, warmup: int, peaks, peak_src, device,
+                         pages_layout: str = "head_major"):
     """The decode workload with its key/value cache in pages of 16 tokens of a
     shared pool, the pages in shuffled order behind each row's block table
-    (sdpa_decode_paged).  Algorithmic bytes: the same K/V bytes as the
+    (sdpa_decode_paged).  ``pages_layout``: "head_major" pools (num_pages,
+    Hkv, 16, E), each head's 16 tokens of a page contiguous; "token_major"
+    (num_pages, 16, Hkv, E).  Algorithmic bytes: the same K/V bytes as the
     contiguous decode (the block table adds 4 bytes per page)."""
     from scaled_dot_product_15_b200 import api, sdpa_decode_paged
 
@@ -406,8 +409,13 @@ def measure_paged_decode(w: W.Workload, steps: int, warmup: int, peaks, peak_src
     perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(w.seed)).to(device)
 
     def pool(t):
-        # (B, Hkv, S, E) -> pages (B*S/16, 16, Hkv, E), page i stored at perm[i]
-        pages = t.transpose(1, 2).reshape(n_pages, PAGE_SIZE, w.Hkv, t.shape[-1])
+        # (B, Hkv, S, E) -> pages, page i stored at perm[i]
+        e = t.shape[-1]
+        if pages_layout == "head_major":
+            pages = t.reshape(w.B, w.Hkv, w.S // PAGE_SIZE, PAGE_SIZE, e).permute(0, 2, 1, 3, 4)
+            pages = pages.reshape(n_pages, w.Hkv, PAGE_SIZE, e)
+        else:
+            pages = t.transpose(1, 2).reshape(n_pages, PAGE_SIZE, w.Hkv, e)
         out = torch.empty_like(pages)
         out[perm] = pages
         return out
@@ -419,10 +427,10 @@ def measure_paged_decode(w: W.Workload, steps: int, warmup: int, peaks, peak_src
     torch.cuda.empty_cache()
     table = perm.to(torch.int32).reshape(w.B, w.S // PAGE_SIZE).contiguous()
     lens = torch.full((w.B,), w.S, dtype=torch.int32, device=device)
-    out, lse = sdpa_decode_paged(q, kp, vp, table, lens)
+    out, lse = sdpa_decode_paged(q, kp, vp, table, lens, pages_layout=pages_layout)
 
     def call():
-        sdpa_decode_paged(q, kp, vp, table, lens, out=out, lse=lse)
+        sdpa_decode_paged(q, kp, vp, table, lens, pages_layout=pages_layout, out=out, lse=lse)
         return api.last_launch_count()
 
     total_ms, kernel_ms, launches = time_device([call], steps, warmup, False)
@@ -437,9 +445,11 @@ def measure_paged_decode(w: W.Workload, steps: int, warmup: int, peaks, peak_src
         "gpu_launches": launches,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 3), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": stored_traffic(w.name + f":paged{PAGE_SIZE}", "decode_paged"),
+                     "traffic": stored_traffic(w.name + f":paged{PAGE_SIZE}"
+                                               + ("" if pages_layout == "head_major" else "_token_major"),
+                                               "decode_paged"),
                      "peak_source": f"of {peak_src}", "algorithmic_per_launch": amount},
-        "note": f"paged cache: pages of {PAGE_SIZE} tokens in shuffled order, one block table per row",
+        "note": f"paged cache: {pages_layout} pages of {PAGE_SIZE} tokens in shuffled order, one block table per row",
     }
     del kp, vp, q, out, lse
     torch.cuda.empty_cache()
@@ -584,6 +594,8 @@ def main():
                     help="time only the workload's backward (gradients) and print one short line (for profilers)")
     ap.add_argument("--bare-paged", action="store_true",
                     help="time only the decode workload over a paged cache and print one short line (for profilers)")
+    ap.add_argument("--pages-layout", default="head_major", choices=["head_major", "token_major"],
+                    help="with --bare-paged: the page pools' layout")
     ap.add_argument("--bare-batch", type=int, default=0,
                     help="with --bare / --bare-paged: use this batch size instead of the workload's "
                          "(smaller profiler captures)")
@@ -614,7 +626,7 @@ def main():
             import dataclasses
 
             w = dataclasses.replace(w, B=args.bare_batch)
-        r = measure_paged_decode(w, args.steps, args.warmup, peaks, peak_src, device)
+        r = measure_paged_decode(w, args.steps, args.warmup, peaks, peak_src, device, args.pages_layout)
         print(json.dumps({"bare_paged": w.name, "ms_per_step": r["ms_per_step"], "path": r["path"],
                           "launches": r["gpu_launches"]}))
         return
@@ -655,11 +667,13 @@ def main():
                 extra[w.name + ":backward"] = {"error": repr(e)}
         for name, ow in W.WORKLOADS.items():
             if ow.L == 1 and ow.mask == "none" and ow.layout != "packed":
-                try:
-                    extra[name + f":paged{PAGE_SIZE}"] = measure_paged_decode(
-                        ow, max(20, args.steps // 4), args.warmup, peaks, peak_src, device)
-                except Exception as e:
-                    extra[name + f":paged{PAGE_SIZE}"] = {"error": repr(e)}
+                for lay, tag in (("head_major", ""), ("token_major", "_token_major")):
+                    key = name + f":paged{PAGE_SIZE}{tag}"
+                    try:
+                        extra[key] = measure_paged_decode(ow, max(20, args.steps // 4), args.warmup, peaks,
+                                                          peak_src, device, lay)
+                    except Exception as e:
+                        extra[key] = {"error": repr(e)}
     if rank == 0 and ws == 1:
         cpu = cpu_baseline(w, args.cpu_seconds)
 

@@ -164,17 +164,13 @@ decode_split_kernel(Params p, int nsplit, int chunk, PagedArgs pg) {
     }
     __syncthreads();
   }
-  // Element offset of key/value token j of this chunk from chunk_base(), or
-  // -1 when its page is not in the pool.
+  // Paged: element offset of key/value token j of this chunk in the pool
+  // (without the head and feature terms), or -1 when its page is not in it.
   auto token_offset = [&](int j, const int64_t* st) -> int64_t {
-    if constexpr (kPaged) {
-      const int tok = s0 + j;
-      const int page = s_page[(tok >> pg.shift) - first_page];
-      if (page < 0) return -1;
-      return (int64_t)page * st[0] + (int64_t)(tok & ((1 << pg.shift) - 1)) * st[2];
-    } else {
-      return (int64_t)(s0 + j) * st[2];
-    }
+    const int tok = s0 + j;
+    const int page = s_page[(tok >> pg.shift) - first_page];
+    if (page < 0) return -1;
+    return (int64_t)page * st[0] + (int64_t)(tok & ((1 << pg.shift) - 1)) * st[2];
   };
   const int gl = lane % G;                 // lane within its group
   const int kg = warp * KPW + lane / G;    // group index
@@ -211,9 +207,14 @@ decode_split_kernel(Params p, int nsplit, int chunk, PagedArgs pg) {
 #pragma unroll
     for (int u = 0; u < kDecUnroll; ++u) {
       const int j = j0 + u * NKG;
-      const int64_t off = j < n ? token_offset(j, p.ks) : -1;
-      if (off >= 0) raw[u] = Vec8<T>::raw(kbase + off);
-      else raw[u] = make_uint4(0, 0, 0, 0);
+      if constexpr (kPaged) {
+        const int64_t off = j < n ? token_offset(j, p.ks) : -1;
+        if (off >= 0) raw[u] = Vec8<T>::raw(kbase + off);
+        else raw[u] = make_uint4(0, 0, 0, 0);
+      } else {
+        if (j < n) raw[u] = Vec8<T>::raw(kbase + (int64_t)(s0 + j) * p.ks[2]);
+        else raw[u] = make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
     for (int u = 0; u < kDecUnroll; ++u) {
@@ -277,9 +278,14 @@ decode_split_kernel(Params p, int nsplit, int chunk, PagedArgs pg) {
 #pragma unroll
     for (int u = 0; u < kDecUnroll; ++u) {
       const int j = j0 + u * NKG;
-      const int64_t off = j < n ? token_offset(j, p.vs) : -1;
-      if (off >= 0) raw[u] = Vec8<T>::raw(vbase + off);
-      else raw[u] = make_uint4(0, 0, 0, 0);
+      if constexpr (kPaged) {
+        const int64_t off = j < n ? token_offset(j, p.vs) : -1;
+        if (off >= 0) raw[u] = Vec8<T>::raw(vbase + off);
+        else raw[u] = make_uint4(0, 0, 0, 0);
+      } else {
+        if (j < n) raw[u] = Vec8<T>::raw(vbase + (int64_t)(s0 + j) * p.vs[2]);
+        else raw[u] = make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
     for (int u = 0; u < kDecUnroll; ++u) {
