@@ -125,9 +125,12 @@ __device__ __forceinline__ float group_reduce_rows(float (&v)[R], int lane, int&
   return v[0];
 }
 
-template <typename T, int E, int R, bool kPaged>
+// kPage: 0 a contiguous cache; 1 a paged one (pages of 1, 2 or 4 tokens);
+// 2 a paged one with pages of 8 tokens or more.
+template <typename T, int E, int R, int kPage>
 __global__ void __launch_bounds__(kDecThreads, (R <= 4 ? 3 : 2))
 decode_split_kernel(Params p, int nsplit, int chunk, PagedArgs pg) {
+  constexpr bool kPaged = kPage != 0;
   constexpr int G = E / 8;              // lanes per key row (16-byte slices)
   constexpr int KPW = 32 / G;           // keys per warp step
   constexpr int NKG = kDecThreads / G;  // lane groups per CTA
@@ -200,43 +203,61 @@ decode_split_kernel(Params p, int nsplit, int chunk, PagedArgs pg) {
 
   // Phase 1: logits.
   const T* kbase = chunk_base(p.k, p.ks);
-  // The loop bound is warp-uniform (the shuffles below need every lane).
-  for (int jb = warp * KPW; jb < n; jb += NKG * kDecUnroll) {
-    const int j0 = jb + lane / G;
-    uint4 raw[kDecUnroll];
+  // Dot products of a key with every query row, reduced over the key's lane
+  // group; the lanes holding a row's sum write its base-2 logit.
+  auto logit = [&](int j, const uint4& raw, bool dropped) {
+    float kf[8];
+    Vec8<T>::cvt(raw, kf);
+    float d[R];
 #pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      const int j = j0 + u * NKG;
-      if constexpr (kPaged) {
-        const int64_t off = j < n ? token_offset(j, p.ks) : -1;
-        if (off >= 0) raw[u] = Vec8<T>::raw(kbase + off);
+    for (int r = 0; r < R; ++r) {
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a = fmaf(qf[r][e], kf[e], a);
+      d[r] = a;
+    }
+    int row;
+    const float full = group_reduce_rows<R, G>(d, gl, row);
+    // lanes holding a replica of the same row: the first one writes
+    if (j < n && (gl % (G / R > 0 ? G / R : 1)) == 0) lg[j * R + row] = dropped ? -INFINITY : full;
+  };
+  if constexpr (kPaged) {
+    // A lane group takes kDecUnroll consecutive keys: with pages of 8 or
+    // more tokens (kPage 2; chunks start at multiples of 8) they share one
+    // page, so the group looks its page up once.  The loop bound is
+    // warp-uniform.
+    for (int it0 = 0; it0 < n; it0 += NKG * kDecUnroll) {
+      const int jg = it0 + kg * kDecUnroll;
+      uint4 raw[kDecUnroll];
+      const int64_t off0 = (kPage == 2 && jg < n) ? token_offset(jg, p.ks) : -1;
+#pragma unroll
+      for (int u = 0; u < kDecUnroll; ++u) {
+        const int j = jg + u;
+        const int64_t off = kPage == 2 ? (off0 >= 0 ? off0 + (int64_t)u * p.ks[2] : -1)
+                                       : (j < n ? token_offset(j, p.ks) : -1);
+        if (j < n && off >= 0) raw[u] = Vec8<T>::raw(kbase + off);
         else raw[u] = make_uint4(0, 0, 0, 0);
-      } else {
+      }
+#pragma unroll
+      for (int u = 0; u < kDecUnroll; ++u) {
+        const int j = jg + u;
+        const bool dropped = kPage == 2 ? off0 < 0 : (j < n && s_page[((s0 + j) >> pg.shift) - first_page] < 0);
+        logit(j, raw[u], dropped);
+      }
+    }
+  } else {
+    // The loop bound is warp-uniform (the shuffles below need every lane).
+    for (int jb = warp * KPW; jb < n; jb += NKG * kDecUnroll) {
+      const int j0 = jb + lane / G;
+      uint4 raw[kDecUnroll];
+#pragma unroll
+      for (int u = 0; u < kDecUnroll; ++u) {
+        const int j = j0 + u * NKG;
         if (j < n) raw[u] = Vec8<T>::raw(kbase + (int64_t)(s0 + j) * p.ks[2]);
         else raw[u] = make_uint4(0, 0, 0, 0);
       }
-    }
 #pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      const int j = j0 + u * NKG;
-      float kf[8];
-      Vec8<T>::cvt(raw[u], kf);
-      float d[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaf(qf[r][e], kf[e], a);
-        d[r] = a;
-      }
-      int row;
-      const float full = group_reduce_rows<R, G>(d, gl, row);
-      // lanes holding a replica of the same row: the first one writes
-      if (j < n && (gl % (G / R > 0 ? G / R : 1)) == 0) {
-        bool dropped = false;  // paged: the key's page is not in the pool
-        if constexpr (kPaged) dropped = s_page[((s0 + j) >> pg.shift) - first_page] < 0;
-        lg[j * R + row] = dropped ? -INFINITY : full;
-      }
+      for (int u = 0; u < kDecUnroll; ++u) logit(j0 + u * NKG, raw[u], false);
     }
   }
   __syncthreads();
@@ -272,33 +293,45 @@ decode_split_kernel(Params p, int nsplit, int chunk, PagedArgs pg) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
   const T* vbase = chunk_base(p.v, p.vs);
-  for (int jb = warp * KPW; jb < n; jb += NKG * kDecUnroll) {
-    const int j0 = jb + lane / G;
-    uint4 raw[kDecUnroll];
+  auto accumulate = [&](int j, const uint4& raw) {
+    if (j >= n) return;
+    float vf[8];
+    Vec8<T>::cvt(raw, vf);
 #pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      const int j = j0 + u * NKG;
-      if constexpr (kPaged) {
-        const int64_t off = j < n ? token_offset(j, p.vs) : -1;
-        if (off >= 0) raw[u] = Vec8<T>::raw(vbase + off);
+    for (int r = 0; r < R; ++r) {
+      const float w = lg[j * R + r];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(w, vf[e], acc[r][e]);
+    }
+  };
+  if constexpr (kPaged) {
+    for (int it0 = 0; it0 < n; it0 += NKG * kDecUnroll) {
+      const int jg = it0 + kg * kDecUnroll;
+      uint4 raw[kDecUnroll];
+      const int64_t off0 = (kPage == 2 && jg < n) ? token_offset(jg, p.vs) : -1;
+#pragma unroll
+      for (int u = 0; u < kDecUnroll; ++u) {
+        const int j = jg + u;
+        const int64_t off = kPage == 2 ? (off0 >= 0 ? off0 + (int64_t)u * p.vs[2] : -1)
+                                       : (j < n ? token_offset(j, p.vs) : -1);
+        if (j < n && off >= 0) raw[u] = Vec8<T>::raw(vbase + off);
         else raw[u] = make_uint4(0, 0, 0, 0);
-      } else {
+      }
+#pragma unroll
+      for (int u = 0; u < kDecUnroll; ++u) accumulate(jg + u, raw[u]);
+    }
+  } else {
+    for (int jb = warp * KPW; jb < n; jb += NKG * kDecUnroll) {
+      const int j0 = jb + lane / G;
+      uint4 raw[kDecUnroll];
+#pragma unroll
+      for (int u = 0; u < kDecUnroll; ++u) {
+        const int j = j0 + u * NKG;
         if (j < n) raw[u] = Vec8<T>::raw(vbase + (int64_t)(s0 + j) * p.vs[2]);
         else raw[u] = make_uint4(0, 0, 0, 0);
       }
-    }
 #pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      const int j = j0 + u * NKG;
-      if (j >= n) continue;
-      float vf[8];
-      Vec8<T>::cvt(raw[u], vf);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float w = lg[j * R + r];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(w, vf[e], acc[r][e]);
-      }
+      for (int u = 0; u < kDecUnroll; ++u) accumulate(j0 + u * NKG, raw[u]);
     }
   }
   __syncthreads();  // weights no longer needed: reuse shared memory
@@ -405,16 +438,18 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int L, int S, int Ev) {
   return (size_t)ns * nrows * ((size_t)Ev + 1) * sizeof(float);
 }
 
-template <typename T, int E, int R, bool kPaged>
+template <typename T, int E, int R, int kPage>
 static cudaError_t launch_decode_t(const Params& p, const PagedArgs& pg, cudaStream_t st, int* launches) {
+  constexpr bool kPaged = kPage != 0;
   const int ns = decode_splits(p.B, p.Hkv, p.S);
-  const int chunk = (p.S + ns - 1) / ns;
+  int chunk = (p.S + ns - 1) / ns;
+  if (kPaged) chunk = (chunk + 7) & ~7;  // chunks start at multiples of 8 tokens (at most 1024 keys still)
   constexpr int G = E / 8;
   constexpr int NKG = kDecThreads / G;
   const size_t smem_lg = (size_t)chunk * R * sizeof(float);
   const size_t smem_red = (size_t)NKG * R * E * sizeof(float);
   const size_t smem = smem_lg > smem_red ? smem_lg : smem_red;
-  auto kern = decode_split_kernel<T, E, R, kPaged>;
+  auto kern = decode_split_kernel<T, E, R, kPage>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid(ns, p.Hkv, p.B);
@@ -431,21 +466,21 @@ static cudaError_t launch_decode_t(const Params& p, const PagedArgs& pg, cudaStr
   return err;
 }
 
-template <typename T, int E, bool kPaged>
+template <typename T, int E, int kPage>
 static cudaError_t launch_decode_e(const Params& p, const PagedArgs& pg, cudaStream_t st, int* launches) {
   const int rows = p.group * p.L;
-  if (rows <= 1) return launch_decode_t<T, E, 1, kPaged>(p, pg, st, launches);
-  if (rows <= 2) return launch_decode_t<T, E, 2, kPaged>(p, pg, st, launches);
-  if (rows <= 4) return launch_decode_t<T, E, 4, kPaged>(p, pg, st, launches);
-  return launch_decode_t<T, E, 8, kPaged>(p, pg, st, launches);
+  if (rows <= 1) return launch_decode_t<T, E, 1, kPage>(p, pg, st, launches);
+  if (rows <= 2) return launch_decode_t<T, E, 2, kPage>(p, pg, st, launches);
+  if (rows <= 4) return launch_decode_t<T, E, 4, kPage>(p, pg, st, launches);
+  return launch_decode_t<T, E, 8, kPage>(p, pg, st, launches);
 }
 
-template <typename T, bool kPaged>
+template <typename T, int kPage>
 static cudaError_t launch_decode_d(const Params& p, const PagedArgs& pg, cudaStream_t st, int* launches) {
   switch (p.E) {
-    case 64: return launch_decode_e<T, 64, kPaged>(p, pg, st, launches);
-    case 128: return launch_decode_e<T, 128, kPaged>(p, pg, st, launches);
-    default: return launch_decode_e<T, 256, kPaged>(p, pg, st, launches);
+    case 64: return launch_decode_e<T, 64, kPage>(p, pg, st, launches);
+    case 128: return launch_decode_e<T, 128, kPage>(p, pg, st, launches);
+    default: return launch_decode_e<T, 256, kPage>(p, pg, st, launches);
   }
 }
 
@@ -469,8 +504,8 @@ bool decode_supported(const Params& p, int dtype) {
 
 cudaError_t launch_decode(const Params& p, int dtype, cudaStream_t st, int* launches) {
   const PagedArgs none = {nullptr, nullptr, 0, 0, 0};
-  if (dtype == SDPA_F16) return launch_decode_d<__half, false>(p, none, st, launches);
-  return launch_decode_d<__nv_bfloat16, false>(p, none, st, launches);
+  if (dtype == SDPA_F16) return launch_decode_d<__half, 0>(p, none, st, launches);
+  return launch_decode_d<__nv_bfloat16, 0>(p, none, st, launches);
 }
 
 // Paged cache: p.k / p.v are the page pools with strides (page, head, token
@@ -478,8 +513,12 @@ cudaError_t launch_decode(const Params& p, int dtype, cudaStream_t st, int* laun
 cudaError_t launch_decode_paged(const Params& p, const int32_t* table, const int32_t* lens, int max_pages,
                                 int num_pages, int page_shift, int dtype, cudaStream_t st, int* launches) {
   const PagedArgs pg = {table, lens, max_pages, num_pages, page_shift};
-  if (dtype == SDPA_F16) return launch_decode_d<__half, true>(p, pg, st, launches);
-  return launch_decode_d<__nv_bfloat16, true>(p, pg, st, launches);
+  if (page_shift >= 3) {
+    if (dtype == SDPA_F16) return launch_decode_d<__half, 2>(p, pg, st, launches);
+    return launch_decode_d<__nv_bfloat16, 2>(p, pg, st, launches);
+  }
+  if (dtype == SDPA_F16) return launch_decode_d<__half, 1>(p, pg, st, launches);
+  return launch_decode_d<__nv_bfloat16, 1>(p, pg, st, launches);
 }
 
 // Reads and clears the decode kernels' error word.  Synchronous.
