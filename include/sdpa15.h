@@ -23,8 +23,8 @@
  *   h / (Hq / Hkv).
  * - lse is float32 for every input dtype (the compute format of the output:
  *   float32 for formats narrower than float32, exactref "logsumexp and its
- *   format").  A row with no kept key has O = 0 and lse = -inf; a NaN input
- *   makes its row NaN (exactref "Special values and dropout").
+ *   format").  A row that sees no key gets O = 0 and lse = -inf; a NaN input
+ *   turns its row into NaN (exactref "Special values and dropout").
  *
  * Memory and threading contract of every entry point below:
  * - All tensor pointers are DEVICE pointers on the current CUDA device.  The

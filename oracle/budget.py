@@ -4,14 +4,14 @@ infrastructure).
 TEST INFRASTRUCTURE ONLY, like the rest of ``oracle/``: only tests use it.
 
 The exactref page "scaled_dot_product_attention" ("Full specification",
-tolerance()) budgets the roundings a computation of the forward makes: the
-score accumulation, the scale factor, one rounding of each logit, the shift by
-the row maximum, exp within a few ulps, the row sum, the final division and
-the rounding to the output dtype; for the logsumexp, log within ulps and the
-rounding of the row maximum plus that logarithm.  It lists what a named
-algorithm adds on top: casting the weights to the input dtype before the
-value product (FlashAttention does this for bf16 and fp16), online-softmax
-rescaling and a reciprocal of the row sum.
+tolerance()) derives its tolerance from the error sources of a forward
+computation: summing the dot products, multiplying by the scale, rounding
+each logit, subtracting the row maximum, the exponential's few-ulp error,
+summing the weights, dividing, and rounding the result to its dtype; and for
+the logsumexp, the logarithm's ulps and the rounding of max + log.  Named
+algorithms add their own sources, listed there too: FlashAttention rounds the
+weights to bf16 / fp16 before multiplying them with V, rescales online and
+multiplies by a reciprocal of the row sum.
 
 ``forward_budget`` turns that list into a first-order bound, element by
 element, for the algorithm the GPU kernels implement, evaluated on the exact
@@ -148,13 +148,14 @@ def backward_budget(
     safety: float = 2.0,
 ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """(tol_dq, tol_dk, tol_dv): per-element first-order bounds for the
-    gradients as the backward kernels compute them (the exactref backward
-    section's list: the forward's scores, scale, logits, shift, exp and row
-    sum; P; the accumulations of dP, D, grad_value, dS K and dS^T Q; the
-    roundings of dS and of the results), with the FlashAttention choices the
-    page names among the algorithms: P recomputed from the forward's fp32
-    logsumexp, P and dS cast to the input dtype before their products, and
-    D_i = grad_i . out_i taken from the forward's output in the input dtype."""
+    gradients as the backward kernels compute them.  The error sources are
+    those the exactref backward section enumerates (recomputing the forward's
+    weights, then summing dP, D and the three gradient products, rounding dS
+    and rounding each result), specialised to the FlashAttention backward
+    the kernels implement: weights rebuilt from the forward's fp32
+    logsumexp, P and dS rounded to the input dtype before they are
+    multiplied, and D_i = grad_i . out_i from the forward's output in the
+    input dtype."""
     q, k, v, g = (_as_f64(x) for x in (query, key, value, grad))
     B, Hq, L, E = q.shape
     _, Hkv, S, _ = k.shape

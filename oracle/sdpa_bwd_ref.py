@@ -17,12 +17,13 @@ the forward (same masks, scale and special-value rules as ``sdpa_ref``),
     grad_query = scale * dS K
     grad_key   = scale * dS^T Q
 
-each summed over the copies that ``enable_gqa`` made of its input (query head
-h reads key/value head h // (Hq // Hkv)).  Non-finite values propagate as IEEE
-arithmetic does: a masked key has P = 0, so an infinite dP there makes D NaN
-(0 * inf); a NaN row of the forward makes every gradient it touches NaN; a row
-with no kept key has P = 0 and contributes 0.  A float mask gets no gradient;
-dropout must be 0.
+where a key/value head shared by several query heads (``enable_gqa``;
+query head h uses key/value head h // (Hq // Hkv)) sums the gradients of all
+of them.  Non-finite values follow IEEE arithmetic: an excluded key has
+P = 0, so an infinite dP under it makes D NaN (zero times infinity); a forward row that
+is NaN spreads NaN to every gradient it feeds; a row that sees no key has
+P = 0 everywhere and adds nothing.  The bias of a float mask is not
+differentiated, and dropout must be 0.
 
 Every value is computed in float64; numpy matmul, exp and sums serve as steps,
 one row block of logits at a time, with no other blocking or reordering.
@@ -46,8 +47,8 @@ __all__ = ["sdpa_backward", "sdpa_backward_packed", "attention_weights"]
 def attention_weights(logits: np.ndarray) -> np.ndarray:
     """Row-wise softmax weights P of a block of logits (rows x S).
 
-    Per exactref "Full specification": a NaN or +inf logit makes the row NaN;
-    a row with no finite logit has weight 0 on every key; otherwise
+    exactref "Full specification": NaN or +inf anywhere in a row makes it
+    NaN; a row without any finite logit gets all-zero weights; otherwise
     P_ij = exp(l_ij - m_i) / sum_j exp(l_ij - m_i)."""
     P = np.zeros_like(logits)
     with np.errstate(invalid="ignore", over="ignore", divide="ignore"):
@@ -77,7 +78,7 @@ def sdpa_backward(
     ``grad`` (B, Hq, L, Ev); the other arguments are the forward's
     (exactref "er.scaled_dot_product_attention.backward")."""
     if dropout_p != 0.0:
-        raise ValueError("dropout is random and has no reference; dropout_p must be 0")
+        raise ValueError("dropout_p must be 0: a random dropout has no deterministic result to check")
     q = _as_f64(query)
     k = _as_f64(key)
     v = _as_f64(value)

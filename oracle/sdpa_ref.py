@@ -11,20 +11,22 @@ What it computes follows the exactref.ai page "scaled_dot_product_attention"
     O = softmax(Q K^T * scale + mask) V      over the key axis
     lse_i = log(sum_j exp(l_ij))             natural log of each row's logits
 
-with ``scale`` defaulting to 1/sqrt(E), applied exactly once; a bool mask keeps
-a key where True, a float mask is added to the scaled scores and -inf removes a
-key; ``is_causal`` keeps key j for query i only when j <= i; with
-``enable_gqa`` the query head axis is a multiple of the key/value head axis and
-query head h reads key/value head h // (Hq // Hkv) (the contiguous grouping of
-the BMGHK layout on the insureai360 xFormers tutorial, section 5
+where ``scale`` is 1/sqrt(E) unless given, and multiplies the raw dot
+products once.  A boolean mask marks the keys a query may see (True = see);
+a floating mask is a bias added after scaling, with -inf meaning the key is
+excluded.  Under ``is_causal`` query i sees keys 0..i only.  With
+``enable_gqa`` several consecutive query heads share one key/value head:
+query head h uses key/value head h // (Hq // Hkv), the contiguous grouping
+of the BMGHK layout (insureai360 xFormers tutorial, section 5
 "Grouped-query attention").
 
-Special values follow the same "Full specification": a logit of +inf or NaN
-makes its row NaN (lse NaN, or +inf when a logit is +inf and none is NaN); a row
-with no finite logit gets weight 0 on every key, so its output is the zero
-weights times V (0, or NaN where V holds a non-finite value: 0 * inf) and its
-lse is -inf; with E = 0 the scores are empty sums, so the logits are the mask
-alone.
+Non-finite values, per the same "Full specification": one NaN or +inf
+among a row's logits turns the whole row into NaN (its lse is NaN, or +inf
+if the row has +inf but no NaN).  When none of a row's logits is finite,
+every weight is zero, the output is those zero weights applied to V (0,
+or NaN where V itself is not finite, since 0 * inf is NaN) and lse is
+-inf.  With E = 0 every dot product is an empty sum (0), so only the mask
+shapes the logits.
 
 Block-diagonal (packed variable-length) attention follows the xFormers
 tutorial, section 4 "Variable-length packed batch": each segment of a packed
@@ -54,8 +56,8 @@ ROW_BLOCK = 256
 def default_scale(E: int) -> float:
     """1/sqrt(E), the page's default for ``scale=None`` (exactref "Arguments").
 
-    For E = 0 the scores are empty sums and the logits are the mask alone, so
-    the scale never multiplies anything; 1.0 is returned as a placeholder."""
+    With E = 0 every dot product is 0 and the scale has nothing to scale;
+    1.0 is returned as a placeholder."""
     if E == 0:
         return 1.0
     return 1.0 / math.sqrt(E)
@@ -72,9 +74,9 @@ def _as_f64(x) -> np.ndarray:
 def _mask_to_bias(attn_mask, shape_bhls: Tuple[int, int, int, int]) -> Optional[np.ndarray]:
     """A bool mask (True keeps) becomes a 0 / -inf bias; a float mask is the bias.
 
-    Follows exactref "Arguments": attn_mask is "a bool mask (True keeps a key)
-    or a float mask added to the scaled scores (-inf removes a key)".  The
-    result is broadcast to (B, Hq, L, S)."""
+    The two mask kinds of exactref "Arguments" (a boolean one marking the
+    visible keys, a floating one added after scaling, -inf excluding the
+    key).  The result is broadcast to (B, Hq, L, S)."""
     if attn_mask is None:
         return None
     if hasattr(attn_mask, "detach"):
@@ -97,9 +99,10 @@ def _softmax_rows(logits: np.ndarray, vals: np.ndarray) -> Tuple[np.ndarray, np.
     """Softmax over the last axis of ``logits`` (rows x S) and the weighted sum
     with ``vals`` (S x Ev); returns (out rows x Ev, lse rows).
 
-    Per exactref "Full specification": a NaN or +inf logit makes the row NaN;
-    a row with no finite logit has weight 0 on every key and lse -inf; else
-    weights are exp(l - max) / sum exp(l - max) and lse = max + log(sum)."""
+    exactref "Full specification": NaN or +inf anywhere in a row makes it
+    NaN; a row without any finite logit gets all-zero weights and lse -inf;
+    otherwise the weights are exp(l - max) / sum exp(l - max) and lse is
+    max + log(sum)."""
     R = logits.shape[0]
     Ev = vals.shape[1]
     out = np.empty((R, Ev), dtype=np.float64)
@@ -145,12 +148,13 @@ def sdpa(
     value (B, Hkv, S, Ev); a 3-D input (B, L, E) is treated as one head.
     Returns ``(out, lse)`` with out (B, Hq, L, Ev) and lse (B, Hq, L).
 
-    ``dropout_p`` must be 0 (exactref "Special values and dropout": dropout is
-    random and has no reference), else ``ValueError``.  Both ``attn_mask`` and
+    ``dropout_p`` must be 0, else ``ValueError``: random dropout has no
+    deterministic result to compare with (exactref "Special values and
+    dropout").  Both ``attn_mask`` and
     ``is_causal`` may be given; each removes keys.
     """
     if dropout_p != 0.0:
-        raise ValueError("dropout is random and has no reference; dropout_p must be 0")
+        raise ValueError("dropout_p must be 0: a random dropout has no deterministic result to check")
     q = _as_f64(query)
     k = _as_f64(key)
     v = _as_f64(value)

@@ -6,10 +6,10 @@ runs in the library's CUDA kernels.  torch provides device memory (outputs and
 the workspace) and the current stream.  There is no fallback: if the library
 is missing or the device is not a B200 the call raises.
 
-Mask arguments are converted to the library's formats here: a bool mask
-(True keeps a key) becomes a float32 0/-inf bias on the device, and a float
-mask of another dtype is cast to float32, as the exactref page's "Arguments"
-define both forms.
+Mask arguments are converted to the library's formats here: a boolean mask
+(True where the key is visible) becomes a float32 bias of 0 and -inf on the
+device, and a floating mask of another dtype is cast to float32 (the two
+mask kinds of the exactref page's "Arguments").
 """
 from __future__ import annotations
 
@@ -179,7 +179,7 @@ def sdpa(
     float32 of shape (B, Hq, L).
     """
     if dropout_p != 0.0:
-        raise ValueError("dropout is random and has no reference; dropout_p must be 0")
+        raise ValueError("dropout_p must be 0: a random dropout has no deterministic result to check")
     if layout == "bmghk":
         return _sdpa_bmghk(query, key, value, attn_mask, is_causal, scale, out, lse)
     lib = load_library()
@@ -285,7 +285,7 @@ def sdpa_backward(
     given the forward's inputs and its outputs ``out`` and ``lse`` (as sdpa()
     returned them); the other arguments are sdpa()'s."""
     if dropout_p != 0.0:
-        raise ValueError("dropout is random and has no reference; dropout_p must be 0")
+        raise ValueError("dropout_p must be 0: a random dropout has no deterministic result to check")
     lib = load_library()
     for t in (query, key, value, out, grad):
         if t.dim() != 4 or not t.is_cuda:

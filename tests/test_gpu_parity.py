@@ -148,8 +148,8 @@ def test_prefill_row_maximum_moves_across_tiles(dt, causal, order):
 
 @pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
 def test_zero_head_size_logits_are_the_mask(dt):
-    """E = 0: the scores are empty sums, so the logits are the mask alone
-    (exactref "Full specification"); with no mask the weights are uniform."""
+    """E = 0: every dot product is 0, so only the mask shapes the logits
+    (exactref "Full specification"); without a mask the weights are uniform."""
     B, H, L, S, Ev = 1, 2, 40, 70, 32
     q = torch.empty((B, H, L, 0), dtype=dt)
     k = torch.empty((B, H, S, 0), dtype=dt)

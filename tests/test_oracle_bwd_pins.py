@@ -3,9 +3,8 @@ mathematics and the pages fix, independently of the oracle's own formulas.
 
 * central finite differences of the forward oracle's loss sum(grad * O): the
   gradient is the derivative of the forward, whatever formula computes it;
-* torch's float64 autograd of its math path, the check the exactref page
-  names for its backward ("Backward checks these gradients against PyTorch's
-  autograd");
+* torch's float64 autograd of its math path, which is what the exactref
+  page's backward section compares its gradients with;
 * invariants: adding one vector to every key of a row's kept set shifts that
   row's logits by a constant, so the key gradients of a head sum to zero;
   the rows of dS sum to zero; grad_value with an all-ones grad is the column

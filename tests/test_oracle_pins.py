@@ -50,8 +50,8 @@ def _qkv(ex):
 
 
 def _assert_rounds_to(out64, printed):
-    """Each printed output is the exact value rounded once to float32; the
-    oracle's float64 value rounded to float32 must land on it (one float32
+    """The page prints float32 results of the exact values; the oracle's
+    float64 value, rounded to float32, must reproduce each one (one float32
     ulp allowed for the double rounding float64 -> float32)."""
     got = _f32(out64)
     want = _f32(printed)
@@ -449,8 +449,8 @@ def test_padding_mask_example():
 
 
 def test_head_dim_zero_logits_are_the_mask():
-    """exactref "Full specification": with E = 0 the scores are empty sums, so
-    the logits are the mask alone."""
+    """exactref "Full specification": with E = 0 every dot product is 0, so
+    only the mask shapes the logits."""
     q = np.zeros((1, 1, 2, 0))
     k = np.zeros((1, 1, 3, 0))
     v = np.array([[[[1.0], [2.0], [4.0]]]])
