@@ -74,6 +74,9 @@ CASES = [
     (torch.float16, 4, 32, 8, 1, 128, 64, 64, 300, [4096, 4095, 65, 64], "token_major"),
     (torch.bfloat16, 1, 32, 8, 1, 128, 16, 1300, 1400, [20000], "head_major"),
     (torch.bfloat16, 2, 4, 1, 1, 64, 2, 600, 1300, [1199, 7], "token_major"),
+    (torch.float16, 2, 8, 1, 1, 256, 4, 300, 700, [1197, 3], "head_major"),     # small pages, 8 rows per head
+    (torch.bfloat16, 3, 32, 8, 1, 128, 4, 400, 1300, [1600, 5, 999], "token_major"),
+    (torch.bfloat16, 2, 16, 2, 1, 128, 8, 200, 450, [1595, 8], "token_major"),  # smallest grouped page, 8 rows
 ]
 
 
