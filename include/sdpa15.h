@@ -17,7 +17,9 @@
  *   of a packed batch to the keys of its own segment (xFormers
  *   BlockDiagonalMask / BlockDiagonalCausalMask, insureai360 tutorial section
  *   4 "Variable-length packed batch"); FLOAT_BIAS adds a float32 bias to the
- *   scaled scores, -inf removing a key.  A bool mask is passed as a 0/-inf bias.
+ *   scaled scores, -inf removing a key; BOOL reads one byte per (b, h, i, j),
+ *   nonzero where query i may see key j, and acts as a 0 / -inf bias (so a
+ *   NaN score under a removed key still makes its row NaN, as a bias would).
  * - GQA (exactref "Arguments", enable_gqa; the BMGHK layout of the tutorial's
  *   section 5): Hq is a multiple of Hkv and query head h reads key/value head
  *   h / (Hq / Hkv).
@@ -64,7 +66,8 @@ typedef enum {
   SDPA_MASK_CAUSAL = 1,
   SDPA_MASK_BLOCK_DIAG = 2,
   SDPA_MASK_BLOCK_DIAG_CAUSAL = 3,
-  SDPA_MASK_FLOAT_BIAS = 4
+  SDPA_MASK_FLOAT_BIAS = 4,
+  SDPA_MASK_BOOL = 5
 } sdpa_mask_kind;
 
 /* Version of this ABI (changes when a signature or an enum changes). */
@@ -108,7 +111,9 @@ size_t sdpa_fwd_workspace_size(int B, int Hq, int Hkv, int L, int S, int E, int 
  *                   grid is sized from it; segments longer than it are an
  *                   error the kernels cannot detect and leave rows unwritten)
  * bias, bias_stride FLOAT_BIAS: device float32 [B, Hq, L, S] with element
- *                   strides (b, h, l, s); 0 broadcasts an axis.  Else ignored.
+ *                   strides (b, h, l, s); 0 broadcasts an axis.  BOOL: device
+ *                   bytes (nonzero = the key is visible) of the same shape,
+ *                   strides in bytes.  Else ignored.
  * workspace         device scratch of sdpa_fwd_workspace_size() bytes (may be
  *                   NULL when that size is 0); its contents need no clearing
  *                   and are garbage afterwards.
@@ -122,7 +127,7 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              const int64_t v_stride[4], const int64_t o_stride[4],
              int has_scale, float scale,
              int mask_kind, const int32_t* cu_seqlens, int n_seqs, int max_seqlen,
-             const float* bias, const int64_t bias_stride[4],
+             const void* bias, const int64_t bias_stride[4],
              int dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
@@ -204,7 +209,7 @@ int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const
              const int64_t dk_stride[4], const int64_t dv_stride[4],
              int has_scale, float scale,
              int mask_kind, const int32_t* cu_seqlens, int n_seqs, int max_seqlen,
-             const float* bias, const int64_t bias_stride[4],
+             const void* bias, const int64_t bias_stride[4],
              int dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*

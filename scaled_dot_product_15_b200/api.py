@@ -6,10 +6,10 @@ runs in the library's CUDA kernels.  torch provides device memory (outputs and
 the workspace) and the current stream.  There is no fallback: if the library
 is missing or the device is not a B200 the call raises.
 
-Mask arguments are converted to the library's formats here: a boolean mask
-(True where the key is visible) becomes a float32 bias of 0 and -inf on the
-device, and a floating mask of another dtype is cast to float32 (the two
-mask kinds of the exactref page's "Arguments").
+Mask arguments are passed in the library's formats: a boolean mask (True
+where the key is visible) as its bytes, a floating mask as float32 (cast
+when it has another dtype) -- the two mask kinds of the exactref page's
+"Arguments".
 """
 from __future__ import annotations
 
@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_PKG, "lib", "libsdpa15.so")
 
 SDPA_OK, SDPA_ERR_INVALID, SDPA_ERR_UNSUPPORTED, SDPA_ERR_CUDA, SDPA_ERR_WORKSPACE = range(5)
 SDPA_F32, SDPA_F16, SDPA_BF16 = 0, 1, 2
-MASK_NONE, MASK_CAUSAL, MASK_BLOCK_DIAG, MASK_BLOCK_DIAG_CAUSAL, MASK_FLOAT_BIAS = range(5)
+MASK_NONE, MASK_CAUSAL, MASK_BLOCK_DIAG, MASK_BLOCK_DIAG_CAUSAL, MASK_FLOAT_BIAS, MASK_BOOL = range(6)
 PLAN_NAMES = {1: "prefill_tcgen05", 2: "decode_split", 3: "simt"}
 
 _DTYPE_CODE = {torch.float32: SDPA_F32, torch.float16: SDPA_F16, torch.bfloat16: SDPA_BF16}
@@ -152,6 +152,22 @@ def _dims(t: torch.Tensor, layout: str):
     return t.shape[0], t.shape[2], t.shape[1], t.shape[3]
 
 
+def _mask_arg(attn_mask: torch.Tensor, dev, B: int, Hq: int, L: int, S: int):
+    """(mask kind, tensor, strides) of an attn_mask for the C ABI: a bool
+    mask goes as bytes (MASK_BOOL, no copy beyond the move to the device), a
+    float mask as float32 (MASK_FLOAT_BIAS); both broadcast to (B, Hq, L, S)
+    with zero strides."""
+    m = attn_mask.to(dev)
+    if m.dtype == torch.bool:
+        kind = MASK_BOOL
+    else:
+        kind = MASK_FLOAT_BIAS
+        if m.dtype != torch.float32:
+            m = m.to(torch.float32)
+    m = m.expand(B, Hq, L, S)
+    return kind, m, _i64x4(m.stride())
+
+
 def sdpa(
     query: torch.Tensor,
     key: torch.Tensor,
@@ -233,15 +249,7 @@ def sdpa(
     elif is_causal:
         mask_kind = MASK_CAUSAL
     elif attn_mask is not None:
-        mask_kind = MASK_FLOAT_BIAS
-        m = attn_mask.to(dev)
-        if m.dtype == torch.bool:
-            m = torch.where(m, 0.0, float("-inf")).to(torch.float32)
-        elif m.dtype != torch.float32:
-            m = m.to(torch.float32)
-        m = m.expand(B, Hq, L, S) if layout == "bhle" else m.expand(B, Hq, L, S)
-        bias_t = m
-        bias_str = _i64x4(m.stride())
+        mask_kind, bias_t, bias_str = _mask_arg(attn_mask, dev, B, Hq, L, S)
 
     qs, ks, vs, os_ = (_i64x4(_strides(t, layout)) for t in (query, key, value, out))
     ws_bytes = lib.sdpa_fwd_workspace_size(B, Hq, Hkv, L, S, E, Ev, mask_kind, dcode)
@@ -322,14 +330,7 @@ def sdpa_backward(
     elif is_causal:
         mask_kind = MASK_CAUSAL
     elif attn_mask is not None:
-        mask_kind = MASK_FLOAT_BIAS
-        m = attn_mask.to(dev)
-        if m.dtype == torch.bool:
-            m = torch.where(m, 0.0, float("-inf")).to(torch.float32)
-        elif m.dtype != torch.float32:
-            m = m.to(torch.float32)
-        bias_t = m.expand(B, Hq, L, S)
-        bias_str = _i64x4(bias_t.stride())
+        mask_kind, bias_t, bias_str = _mask_arg(attn_mask, dev, B, Hq, L, S)
     dq, dk, dv = torch.empty_like(query), torch.empty_like(key), torch.empty_like(value)
     strides = [_i64x4(_strides(t, layout)) for t in (query, key, value, out, grad, dq, dk, dv)]
     ws_bytes = lib.sdpa_bwd_workspace_size(B, Hq, Hkv, L, S, E, Ev, mask_kind, dcode)

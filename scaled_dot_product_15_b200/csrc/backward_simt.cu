@@ -140,6 +140,10 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkdv_kernel(Params p, BwdP
     const float* lseb = p.lse + ((int64_t)b * p.Hq + h) * p.L;
     const float* Db = g.D + ((int64_t)b * p.Hq + h) * p.L;
     const float* biasb = (p.mask == SDPA_MASK_FLOAT_BIAS) ? p.bias + b * p.bs[0] + h * p.bs[1] : nullptr;
+    // BOOL: bytes (nonzero = visible) in the bias pointer, a 0 / -inf bias
+    const unsigned char* boolb = (p.mask == SDPA_MASK_BOOL)
+                                     ? reinterpret_cast<const unsigned char*>(p.bias) + b * p.bs[0] + h * p.bs[1]
+                                     : nullptr;
     for (int i0 = blo; i0 < bhi; i0 += kBwdTile) {
       const int ni = min(kBwdTile, bhi - i0);
       __syncthreads();  // previous tile consumed
@@ -170,6 +174,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkdv_kernel(Params p, BwdP
         dpd = warp_sum(dpd);
         float logit = p.E == 0 ? 0.f : dot * p.scale;  // E = 0: empty sums
         if (biasb) logit += __ldg(biasb + (int64_t)i * p.bs[2] + (int64_t)j * p.bs[3]);
+        if (boolb) logit += __ldg(boolb + (int64_t)i * p.bs[2] + (int64_t)j * p.bs[3]) ? 0.f : -INFINITY;
         const float pij = weight(logit, s_lse[ii]);
         const float ds = pij * (dpd - s_D[ii]);
 #pragma unroll
@@ -221,6 +226,11 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dq_kernel(Params p, BwdPar
   const float* biasp = (p.mask == SDPA_MASK_FLOAT_BIAS && row_ok)
                            ? p.bias + b * p.bs[0] + h * p.bs[1] + (int64_t)i * p.bs[2]
                            : nullptr;
+  // BOOL: bytes (nonzero = visible) in the bias pointer, a 0 / -inf bias
+  const unsigned char* boolp = (p.mask == SDPA_MASK_BOOL && row_ok)
+                                   ? reinterpret_cast<const unsigned char*>(p.bias) + b * p.bs[0] + h * p.bs[1] +
+                                         (int64_t)i * p.bs[2]
+                                   : nullptr;
   float qr[kBwdMaxPL], gr[kBwdMaxPL], dq[kBwdMaxPL];
 #pragma unroll
   for (int t = 0; t < kBwdMaxPL; ++t) {
@@ -255,6 +265,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dq_kernel(Params p, BwdPar
       dpd = warp_sum(dpd);
       float logit = p.E == 0 ? 0.f : dot * p.scale;  // E = 0: empty sums
       if (biasp) logit += __ldg(biasp + (int64_t)j * p.bs[3]);
+      if (boolp) logit += __ldg(boolp + (int64_t)j * p.bs[3]) ? 0.f : -INFINITY;
       const float ds = weight(logit, lse) * (dpd - Di);
 #pragma unroll
       for (int t = 0; t < kBwdMaxPL; ++t) {

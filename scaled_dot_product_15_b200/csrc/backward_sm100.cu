@@ -823,7 +823,7 @@ bool backward_sm100_supported(const Params& p, const BwdParams& g, int dtype) {
   using tmahost::strides_ok;
   if (dtype != SDPA_F16 && dtype != SDPA_BF16) return false;
   if (p.E != p.Ev || (p.E != 64 && p.E != 96 && p.E != 128)) return false;
-  if (p.mask == SDPA_MASK_FLOAT_BIAS) return false;
+  if (p.mask == SDPA_MASK_FLOAT_BIAS || p.mask == SDPA_MASK_BOOL) return false;
   if (!(p.scale > 0.f) || !isfinite(p.scale)) return false;
   if (p.L < 1 || p.S < 1) return false;
   const bool varlen = p.mask == SDPA_MASK_BLOCK_DIAG || p.mask == SDPA_MASK_BLOCK_DIAG_CAUSAL;

@@ -33,7 +33,8 @@ thread_local int t_last_launches = 0;
 enum Plan { kPlanPrefill = 1, kPlanDecode = 2, kPlanSimt = 3 };
 
 bool valid_dtype(int d) { return d == SDPA_F32 || d == SDPA_F16 || d == SDPA_BF16; }
-bool valid_mask(int m) { return m >= SDPA_MASK_NONE && m <= SDPA_MASK_FLOAT_BIAS; }
+bool valid_mask(int m) { return m >= SDPA_MASK_NONE && m <= SDPA_MASK_BOOL; }
+bool has_bias(int m) { return m == SDPA_MASK_FLOAT_BIAS || m == SDPA_MASK_BOOL; }
 
 // Checks shapes and strides that do not need device data.  Returns SDPA_OK or
 // an error status.
@@ -68,6 +69,7 @@ void fill_params(Params& p, const void* q, const void* k, const void* v, void* o
 }
 
 int choose_plan(const Params& p, int dtype) {
+  if (p.mask == SDPA_MASK_BOOL) return kPlanSimt;  // bool masks run on the general kernels only
   if (dtype != SDPA_F32) {
     if (decode_supported(p, dtype)) return kPlanDecode;
     if (prefill_supported(p, dtype)) return kPlanPrefill;
@@ -148,7 +150,7 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              int Hkv, int L, int S, int E, int Ev, const int64_t q_stride[4],
              const int64_t k_stride[4], const int64_t v_stride[4], const int64_t o_stride[4],
              int has_scale, float scale, int mask_kind, const int32_t* cu_seqlens, int n_seqs,
-             int max_seqlen, const float* bias, const int64_t bias_stride[4], int dtype,
+             int max_seqlen, const void* bias, const int64_t bias_stride[4], int dtype,
              void* workspace, size_t workspace_bytes, void* stream) {
   t_last_launches = 0;
   int st = check_shapes(B, Hq, Hkv, L, S, E, Ev, q_stride, k_stride, v_stride, o_stride, mask_kind, dtype);
@@ -161,7 +163,7 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   if (mask_kind == SDPA_MASK_BLOCK_DIAG || mask_kind == SDPA_MASK_BLOCK_DIAG_CAUSAL) {
     if (!cu_seqlens || n_seqs < 1 || max_seqlen < 1) return SDPA_ERR_INVALID;
   }
-  if (mask_kind == SDPA_MASK_FLOAT_BIAS) {
+  if (has_bias(mask_kind)) {
     if (!bias || !bias_stride) return SDPA_ERR_INVALID;
     for (int d = 0; d < 4; ++d)
       if (bias_stride[d] < 0) return SDPA_ERR_INVALID;
@@ -176,8 +178,10 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   p.cu = cu_seqlens;
   p.n_seqs = n_seqs;
   p.max_seqlen = max_seqlen;
-  if (mask_kind == SDPA_MASK_FLOAT_BIAS) {
-    p.bias = bias;
+  if (has_bias(mask_kind)) {
+    // BOOL: the byte mask travels in the bias pointer; the kernels read it
+    // as bytes when p.mask says so.
+    p.bias = static_cast<const float*>(bias);
     for (int d = 0; d < 4; ++d) p.bs[d] = bias_stride[d];
   }
   p.ws = workspace;
@@ -216,7 +220,7 @@ int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const
              const int64_t v_stride[4], const int64_t o_stride[4], const int64_t do_stride[4],
              const int64_t dq_stride[4], const int64_t dk_stride[4], const int64_t dv_stride[4],
              int has_scale, float scale, int mask_kind, const int32_t* cu_seqlens, int n_seqs,
-             int max_seqlen, const float* bias, const int64_t bias_stride[4], int dtype,
+             int max_seqlen, const void* bias, const int64_t bias_stride[4], int dtype,
              void* workspace, size_t workspace_bytes, void* stream) {
   t_last_launches = 0;
   int st = check_shapes(B, Hq, Hkv, L, S, E, Ev, q_stride, k_stride, v_stride, o_stride, mask_kind, dtype);
@@ -235,7 +239,7 @@ int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const
   if (mask_kind == SDPA_MASK_BLOCK_DIAG || mask_kind == SDPA_MASK_BLOCK_DIAG_CAUSAL) {
     if (!cu_seqlens || n_seqs < 1 || max_seqlen < 1) return SDPA_ERR_INVALID;
   }
-  if (mask_kind == SDPA_MASK_FLOAT_BIAS) {
+  if (has_bias(mask_kind)) {
     if (!bias || !bias_stride) return SDPA_ERR_INVALID;
     for (int d = 0; d < 4; ++d)
       if (bias_stride[d] < 0) return SDPA_ERR_INVALID;
@@ -254,8 +258,10 @@ int sdpa_bwd(const void* q, const void* k, const void* v, const void* out, const
   p.cu = cu_seqlens;
   p.n_seqs = n_seqs;
   p.max_seqlen = max_seqlen;
-  if (mask_kind == SDPA_MASK_FLOAT_BIAS) {
-    p.bias = bias;
+  if (has_bias(mask_kind)) {
+    // BOOL: the byte mask travels in the bias pointer; the kernels read it
+    // as bytes when p.mask says so.
+    p.bias = static_cast<const float*>(bias);
     for (int d = 0; d < 4; ++d) p.bs[d] = bias_stride[d];
   }
   BwdParams g;

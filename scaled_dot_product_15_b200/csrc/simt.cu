@@ -70,9 +70,14 @@ simt_attention_kernel(Params p) {
   float m = -INFINITY, lsum = 0.f;
   bool bad_nan = false, bad_pinf = false;
 
+  // FLOAT_BIAS: float32 bias; BOOL: bytes (nonzero = visible) in the same
+  // pointer, applied as a 0 / -inf bias.
   const float* biasp = nullptr;
+  const unsigned char* boolp = nullptr;
   if (p.mask == SDPA_MASK_FLOAT_BIAS && row_ok)
     biasp = p.bias + b * p.bs[0] + h * p.bs[1] + (int64_t)i * p.bs[2];
+  if (p.mask == SDPA_MASK_BOOL && row_ok)
+    boolp = reinterpret_cast<const unsigned char*>(p.bias) + b * p.bs[0] + h * p.bs[1] + (int64_t)i * p.bs[2];
 
   for (int j0 = blo; j0 < bhi; j0 += kSimtKeys) {
     const int nk = min(kSimtKeys, bhi - j0);
@@ -98,6 +103,7 @@ simt_attention_kernel(Params p) {
       dot = warp_sum(dot);
       float logit = (p.E == 0) ? 0.f : dot * p.scale;
       if (biasp) logit = logit + __ldg(biasp + (int64_t)j * p.bs[3]);
+      if (boolp) logit = logit + (__ldg(boolp + (int64_t)j * p.bs[3]) ? 0.f : -INFINITY);
       if (isnan(logit)) { bad_nan = true; continue; }
       if (logit == INFINITY) { bad_pinf = true; continue; }
       if (logit == -INFINITY) continue;  // removed key: weight 0

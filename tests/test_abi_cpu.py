@@ -69,6 +69,8 @@ def test_host_side_rejections():
     assert _call(mask=api.MASK_BLOCK_DIAG, B=2) == api.SDPA_ERR_INVALID
     assert _call(mask=api.MASK_BLOCK_DIAG) == api.SDPA_ERR_INVALID  # no cu_seqlens
     assert _call(mask=api.MASK_FLOAT_BIAS) == api.SDPA_ERR_INVALID  # no bias
+    assert _call(mask=api.MASK_BOOL) == api.SDPA_ERR_INVALID       # no byte mask
+    assert _call(mask=6) == api.SDPA_ERR_INVALID                    # unknown mask kind
     assert _call(scale=float("nan")) == api.SDPA_ERR_INVALID
     assert _call(ptr=None) == api.SDPA_ERR_INVALID
     assert _call(B=0) == api.SDPA_OK                            # empty problem: nothing to do
@@ -106,6 +108,7 @@ def test_dispatch_plan():
     assert _plan(64, 32, 8, 1, 16384, 128, 128, 0, api.SDPA_BF16) == 2       # GQA decode
     assert _plan(64, 32, 8, 1, 16384, 128, 128, 0, api.SDPA_BF16, align=2) == 3  # unaligned
     assert _plan(1, 2, 2, 64, 64, 48, 48, api.MASK_FLOAT_BIAS, api.SDPA_F16) == 3
+    assert _plan(1, 2, 2, 256, 256, 128, 128, api.MASK_BOOL, api.SDPA_BF16) == 3  # bool masks: general kernels
     assert _plan(1, 3, 2, 64, 64, 64, 64, 0, api.SDPA_F16) == -api.SDPA_ERR_INVALID
 
 

@@ -420,3 +420,34 @@ def test_full_bf16_gqa_decode_sampled():
         ro, rl = ref_sdpa(qs, ks, vs, enable_gqa=True)
         assert_close(out[b, kvh * g:(kvh + 1) * g][None], lse[b, kvh * g:(kvh + 1) * g][None], ro, rl,
                      w.torch_dtype, f"decode b={b} kvh={kvh}")
+
+
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
+def test_native_bool_mask_matches_its_bias_form(dt):
+    """A bool mask passed natively (one byte per element, broadcast over
+    heads) gives the same result as the same mask written as a 0 / -inf
+    float bias, and both match the oracle; a NaN score under a removed key
+    still makes its row NaN, as a bias would."""
+    from scaled_dot_product_15_b200 import plan
+
+    B, Hq, Hkv, L, S, E = 2, 4, 2, 70, 90, 64
+    q, k, v = _rand((B, Hq, L, E), 521, dt), _rand((B, Hkv, S, E), 522, dt), _rand((B, Hkv, S, E), 523, dt)
+    m = torch.rand((B, 1, L, S), generator=torch.Generator().manual_seed(524)) > 0.4
+    m[1, 0, 11] = False                     # a row with no visible key
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    assert plan(qd, kd, vd, mask_kind=5) == "simt"
+    out, lse = _sdpa(qd, kd, vd, attn_mask=m.to(DEV), enable_gqa=True)
+    bias = torch.where(m, 0.0, float("-inf"))
+    ob, lb = _sdpa(qd, kd, vd, attn_mask=bias.to(DEV), enable_gqa=True)
+    assert torch.equal(out, ob) and torch.equal(lse, lb)
+    ro, rl = ref_sdpa(q, k, v, attn_mask=m, enable_gqa=True)
+    assert_close(out, lse, ro, rl, dt, "native bool mask")
+    assert (out[1, :, 11] == 0).all() and torch.isneginf(lse[1, :, 11]).all()
+    qn = q.clone()
+    qn[0, 0, 3, 0] = float("nan")           # NaN in every score of row 3 of head 0
+    m2 = m.clone()
+    m2[0, 0, 3, :5] = False
+    out, lse = _sdpa(qn.to(DEV), kd, vd, attn_mask=m2.to(DEV), enable_gqa=True)
+    ro, rl = ref_sdpa(qn, k, v, attn_mask=m2, enable_gqa=True)
+    assert_close(out, lse, ro, rl, dt, "NaN under removed keys")
+    assert torch.isnan(out[0, 0, 3]).all()
