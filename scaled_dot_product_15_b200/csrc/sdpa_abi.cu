@@ -27,7 +27,7 @@ using namespace sdpa15;
 
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 thread_local int t_last_launches = 0;
 
 enum Plan { kPlanPrefill = 1, kPlanDecode = 2, kPlanSimt = 3 };
