@@ -394,6 +394,29 @@ def measure_backward(w: W.Workload, steps: int, warmup: int, peaks, peak_src, de
 PAGE_SIZE = 16
 
 
+def paged_cache(k, v, page_size: int, pages_layout: str, seed: int):
+    """A contiguous (B, Hkv, S, E) cache rewritten as a page pool: pages of
+    ``page_size`` tokens, page i of the identity order stored at pool slot
+    perm[i] for a seeded permutation, and the block table that undoes it.
+    Returns (k_pages, v_pages, block_table int32 (B, S/page_size))."""
+    B, Hkv, S, _ = k.shape
+    n_pages = B * S // page_size
+    perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(seed)).to(k.device)
+
+    def pool(t):
+        e = t.shape[-1]
+        if pages_layout == "head_major":
+            pages = t.reshape(B, Hkv, S // page_size, page_size, e).permute(0, 2, 1, 3, 4)
+            pages = pages.reshape(n_pages, Hkv, page_size, e)
+        else:
+            pages = t.transpose(1, 2).reshape(n_pages, page_size, Hkv, e)
+        out = torch.empty_like(pages)
+        out[perm] = pages
+        return out
+
+    return pool(k), pool(v), perm.to(torch.int32).reshape(B, S // page_size).contiguous()
+
+
 def measure_paged_decode(w: W.Workload, steps: int, warmup: int, peaks, peak_src, device,
                          pages_layout: str = "head_major"):
     """The decode workload with its key/value cache in pages of 16 tokens of a
@@ -405,27 +428,9 @@ def measure_paged_decode(w: W.Workload, steps: int, warmup: int, peaks, peak_src
     from scaled_dot_product_15_b200 import api, sdpa_decode_paged
 
     q, k, v = W.make_inputs(w, device)
-    n_pages = w.B * w.S // PAGE_SIZE
-    perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(w.seed)).to(device)
-
-    def pool(t):
-        # (B, Hkv, S, E) -> pages, page i stored at perm[i]
-        e = t.shape[-1]
-        if pages_layout == "head_major":
-            pages = t.reshape(w.B, w.Hkv, w.S // PAGE_SIZE, PAGE_SIZE, e).permute(0, 2, 1, 3, 4)
-            pages = pages.reshape(n_pages, w.Hkv, PAGE_SIZE, e)
-        else:
-            pages = t.transpose(1, 2).reshape(n_pages, PAGE_SIZE, w.Hkv, e)
-        out = torch.empty_like(pages)
-        out[perm] = pages
-        return out
-
-    kp = pool(k)
-    del k
-    vp = pool(v)
-    del v
+    kp, vp, table = paged_cache(k, v, PAGE_SIZE, pages_layout, w.seed)
+    del k, v
     torch.cuda.empty_cache()
-    table = perm.to(torch.int32).reshape(w.B, w.S // PAGE_SIZE).contiguous()
     lens = torch.full((w.B,), w.S, dtype=torch.int32, device=device)
     out, lse = sdpa_decode_paged(q, kp, vp, table, lens, pages_layout=pages_layout)
 

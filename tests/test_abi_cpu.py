@@ -189,3 +189,16 @@ def test_paged_decode_without_gpu_is_unsupported():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _paged() == api.SDPA_ERR_UNSUPPORTED
+
+
+def test_mask_arguments_are_marshalled_without_conversion_of_bool_masks():
+    import torch
+
+    m = torch.rand(5, 7) > 0.5
+    kind, t, st = api._mask_arg(m, torch.device("cpu"), 2, 3, 5, 7)
+    assert kind == api.MASK_BOOL and t.dtype == torch.bool and t.data_ptr() == m.data_ptr()
+    assert tuple(st) == (0, 0, 7, 1) and t.shape == (2, 3, 5, 7)      # broadcast, byte strides
+    f = torch.randn(2, 1, 5, 7, dtype=torch.float16)
+    kind, t, st = api._mask_arg(f, torch.device("cpu"), 2, 3, 5, 7)
+    assert kind == api.MASK_FLOAT_BIAS and t.dtype == torch.float32
+    assert tuple(st) == (35, 0, 7, 1)
