@@ -23,9 +23,9 @@
  * - GQA (exactref "Arguments", enable_gqa; the BMGHK layout of the tutorial's
  *   section 5): Hq is a multiple of Hkv and query head h reads key/value head
  *   h / (Hq / Hkv).
- * - lse is float32 for every input dtype (the compute format of the output:
- *   float32 for formats narrower than float32, exactref "logsumexp and its
- *   format").  A row that sees no key gets O = 0 and lse = -inf; a NaN input
+ * - lse is float32 for every input dtype: exactref "logsumexp and its
+ *   format" computes it in float32 for the 16-bit formats and in the input's
+ *   own format otherwise, which here is float32 too.  A row that sees no key gets O = 0 and lse = -inf; a NaN input
  *   turns its row into NaN (exactref "Special values and dropout").
  *
  * Memory and threading contract of every entry point below:

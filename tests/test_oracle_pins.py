@@ -387,8 +387,8 @@ def test_row_bias_shift_and_value_linearity():
 
 
 def test_nan_row(ex):
-    """exactref "Special values and dropout": one query that holds a NaN gives
-    a NaN row ([[nan, nan]]); the other rows are unaffected."""
+    """exactref "Special values and dropout": a query containing a NaN makes
+    its own output row NaN ([[nan, nan]]) and leaves the other rows alone."""
     _, k, v = _qkv(ex)
     out, lse = sdpa(np.array([[[np.nan, 0.0]]], dtype=np.float32), k, v)
     assert np.isnan(out).all() and out.shape == (1, 1, 2)
